@@ -1,0 +1,163 @@
+/*
+ * vdn.h -- C ABI of libvdn, the sm_100a (B200) implementation of the Video
+ * DeltaNet hybrid attention forward for video-to-video interactions.
+ *
+ * Source of every operation: "Video DeltaNet: A Video-Native Hybrid Attention
+ * for Livestream Video Generation" (Xi et al.):
+ *   - Softmax branch: the "Nearby frames ..." paragraph of the method (exact
+ *     Softmax inside a chunk-aligned window of 2*window_radius+1 chunks, plus
+ *     the two boundary anchors: every frame sees all tokens of the first and
+ *     last latent frame, and those two frames see the whole clip; a key frame
+ *     counts once).
+ *   - Linear branch: the "Bidirectional linear attention ..." paragraph (a
+ *     forward and a reverse scan over the frames outside the query's window,
+ *     anchors excluded, both initialised from a text-summary state, readouts
+ *     added; a channel-wise decay bridge across the skipped window span) and
+ *     the Video Delta Attention paragraphs (per-frame joint update
+ *     S_t = (I + A_t)^-1 (Diag(alpha_t) S_{t-1} + W_t), A_t = beta_t K_t^T K_t,
+ *     W_t = beta_t K_t^T V_t, solved in key-channel space, FP32 state).
+ *   - Output: the "Both branches receive ..." paragraph (sigmoid gate on the
+ *     Softmax readout, RMS norm + sigmoid gate on the linear readout, two
+ *     separate output projections whose results are added).
+ *   - Implementation section ("Chunk-wise scans", "Small-matrix inverse"):
+ *     per-frame affine transitions composed per chunk and scanned in both
+ *     directions; only chunk-boundary states are kept.
+ *
+ * Conventions shared by every entry point
+ *   - Sizes: L = T*N video tokens per batch item, token index t*N + n
+ *     (frame-major).  n_chunks = ceil(T / chunk).  Anchors = frames {0, T-1}.
+ *   - Layouts (row-major, innermost last):
+ *       q, k, v            [B, L, H, d]      dtype params.dtype
+ *       text_k, text_v     [B, n_text, H, d] dtype params.dtype
+ *       beta               [B, H, 1+T]       float32; [.,.,0] is the text frame
+ *       alpha              [B, H, T, d_k]    float32 in [0,1], or NULL (= 1)
+ *       W_o_soft, W_o_lin  [H*d_v, D_out]    dtype params.dtype; y = x W
+ *       gates              [2, B, L, H, d_v] dtype params.dtype, post-sigmoid;
+ *                                            [0] Softmax gate, [1] linear gate
+ *       out                [B, L, D_out]     dtype params.out_dtype
+ *   - Ownership: the caller owns every buffer (device memory unless stated).
+ *     The library never allocates or frees device memory; all scratch comes
+ *     from the caller's workspace (size from vdn_workspace_bytes).
+ *   - Alignment: every pointer must be 16-byte aligned.
+ *   - Asynchrony: compute entry points validate arguments on the host, then
+ *     enqueue kernels on `stream` and return without synchronising.  VDN_OK
+ *     means "enqueued".  Device-side conditions (a bounded wait that expired,
+ *     a value outside the range of an internal fp16 operand) are recorded in
+ *     a status word inside the workspace; read it with vdn_device_status.
+ *   - Errors: a failed validation returns before any launch and leaves every
+ *     output untouched.  No exceptions cross the ABI.  The library keeps no
+ *     global state except a per-device attribute cache; calls on different
+ *     streams with different workspaces may run concurrently.
+ *   - Supported: d_k == d_v in {32, 64, 128} (any d with VDN_FLAG_SIMT up to
+ *     128), chunk >= 1, window_radius >= 0, T >= 1, N >= 1, n_text >= 0,
+ *     D_out a multiple of 8.  Tensor-core kernels serve dtype BF16 with
+ *     d in {64, 128}; every other case runs the exact-FP32 CUDA-core kernels.
+ */
+#ifndef VDN_H_
+#define VDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VDN_ABI_VERSION 1
+
+typedef enum vdn_status {
+  VDN_OK = 0,
+  VDN_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, bad enum/flag */
+  VDN_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  VDN_ERR_DTYPE = 3,       /* unsupported dtype combination */
+  VDN_ERR_ALIGNMENT = 4,   /* a pointer is not 16-byte aligned */
+  VDN_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than required */
+  VDN_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
+  VDN_ERR_TIMEOUT = 7,     /* a bounded device-side wait expired */
+  VDN_ERR_UNSUPPORTED = 8, /* valid request that this build does not serve */
+  VDN_ERR_RANGE = 9        /* an input value overflowed an internal fp16 operand */
+} vdn_status;
+
+typedef enum vdn_dtype { VDN_F32 = 0, VDN_BF16 = 1 } vdn_dtype;
+
+/* Binary-compatible with cudaStream_t / CUstream; NULL = legacy default stream. */
+typedef struct CUstream_st *vdn_stream_t;
+
+/* params.flags */
+#define VDN_FLAG_TEXT_FULL (1u << 0) /* both scans start from S_text (not S_text/2) */
+#define VDN_FLAG_SIMT (1u << 1)      /* force the exact-FP32 CUDA-core kernels */
+
+typedef struct vdn_params {
+  int B;             /* batch */
+  int H;             /* heads */
+  int T;             /* latent frames */
+  int N;             /* tokens per frame */
+  int d_k, d_v;      /* head dims (must be equal) */
+  int n_text;        /* text tokens summarised into the initial state */
+  int D_out;         /* output width of both projections */
+  int chunk;         /* frames per chunk (5 on the pages: one VAE temporal unit) */
+  int window_radius; /* chunks on each side of the query chunk (1 on the pages) */
+  vdn_dtype dtype;     /* q, k, v, text_k, text_v, W_o_*, gates */
+  vdn_dtype out_dtype; /* out */
+  float softmax_scale; /* 0 => 1/sqrt(d_k) */
+  float rms_eps;       /* epsilon of the linear-readout RMS norm (pages: unstated; 1e-6) */
+  unsigned flags;      /* VDN_FLAG_* */
+} vdn_params;
+
+/* ABI version of the loaded library (VDN_ABI_VERSION). */
+int vdn_abi_version(void);
+
+/* Static string for a status code; never NULL. */
+const char *vdn_status_string(vdn_status s);
+
+/* Fills `p` with the pages' defaults for the given sizes: chunk 5,
+ * window_radius 1, D_out = H*d, softmax_scale 0, rms_eps 1e-6, flags 0. */
+vdn_status vdn_params_init(vdn_params *p, int B, int H, int T, int N, int d,
+                           int n_text, vdn_dtype dtype);
+
+/* Workspace bytes needed by vdn_hybrid_attn_fwd, vdn_hybrid_attn_branches
+ * and vdn_vda_boundary_states for these params (one size serves all three).
+ * Host only; validates `p` like the compute calls. */
+vdn_status vdn_workspace_bytes(const vdn_params *p, size_t *bytes);
+
+/* The whole hybrid attention forward:
+ *   o_s = window+anchor Softmax(q, k, v)                          [B,L,H,d_v]
+ *   o_l = q^T S_fwd + q^T S_rev (VDA scans, text-initialised)      [B,L,H,d_v]
+ *   out = concat_h(g_s * o_s) W_o_soft + concat_h(g_l * RMS(o_l)) W_o_lin
+ * alpha may be NULL (no decay).  n_text may be 0 (text_k/text_v may then be
+ * NULL; S_text = 0).  Everything else is required. */
+vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const void *k,
+                               const void *v, const float *beta, const float *alpha,
+                               const void *text_k, const void *text_v,
+                               const void *W_o_soft, const void *W_o_lin,
+                               const void *gates, void *out, void *workspace,
+                               size_t workspace_bytes, vdn_stream_t stream);
+
+/* The two branch readouts before gating and projection, float32
+ * [B, L, H, d_v]: o_soft = Softmax branch, o_lin = linear branch before its
+ * RMS norm.  Either output pointer may be NULL to skip that branch. */
+vdn_status vdn_hybrid_attn_branches(const vdn_params *p, const void *q, const void *k,
+                                    const void *v, const float *beta, const float *alpha,
+                                    const void *text_k, const void *text_v,
+                                    float *o_soft, float *o_lin, void *workspace,
+                                    size_t workspace_bytes, vdn_stream_t stream);
+
+/* The chunk-boundary states of the VDA scans, float32 [B, H, n_chunks, d_k, d_v]:
+ * F[c] = forward state read by query chunk c (after every frame before its
+ * window), G[c] = reverse state (after every frame after its window), before
+ * the per-frame decay bridge.  Either output may be NULL. */
+vdn_status vdn_vda_boundary_states(const vdn_params *p, const void *k, const void *v,
+                                   const float *beta, const float *alpha,
+                                   const void *text_k, const void *text_v, float *F,
+                                   float *G, void *workspace, size_t workspace_bytes,
+                                   vdn_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device status word that
+ * the last calls on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
+ * VDN_ERR_RANGE).  `workspace` must be the one passed to those calls. */
+vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDN_H_ */

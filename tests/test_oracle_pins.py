@@ -1,0 +1,364 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a textbook
+routine (token-level delta rule, least squares, dense softmax), a closed form,
+an invariant stated on the pages, or brute-force enumeration on tiny inputs.
+The pages print no worked numeric example (every displayed equation was lost
+in extraction), so no printed values are available to pin.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import scipy.special
+
+from oracle import vdn_oracle as O
+
+rng_global = np.random.default_rng(0)
+
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def _delta_rule_token(S, k, v, beta_eff):
+    """Textbook token-level delta rule (Gated DeltaNet form, without decay):
+    read the prediction S^T k, write beta_eff * k (v - S^T k)^T."""
+    pred = S.T @ k
+    return S + beta_eff * np.outer(k, v - pred)
+
+
+# --- Video Delta Attention frame update --------------------------------------
+
+@pytest.mark.parametrize("seed", range(5))
+def test_n1_reduces_to_token_delta_rule(seed):
+    """With one token per frame, the VDA update equals the token-level delta
+    rule with the effective write strength beta/(1 + beta ||k||^2)
+    (Sherman-Morrison on (I + beta k k^T)^-1)."""
+    rng = np.random.default_rng(seed)
+    dk, dv = 6, 5
+    S = rng.normal(size=(dk, dv))
+    k = rng.normal(size=dk)          # not unit: exercises the ||k||^2 term
+    v = rng.normal(size=dv)
+    beta = rng.uniform(0.05, 3.0)
+    alpha = rng.uniform(0.5, 1.0, size=dk)
+    got = O.vda_update(S, k[None, :], v[None, :], beta, alpha)
+    S_dec = alpha[:, None] * S
+    want = _delta_rule_token(S_dec, k, v, beta / (1.0 + beta * k @ k))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_joint_objective_least_squares(seed):
+    """The frame update is the minimiser of 1/2||S - S~||^2 +
+    1/2 sum_i beta ||S^T k_i - v_i||^2; solve the stacked least-squares system
+    [I; sqrt(beta) K] S = [S~; sqrt(beta) V] with a generic routine."""
+    rng = np.random.default_rng(100 + seed)
+    dk, dv, n = 7, 4, 11
+    S_prev = rng.normal(size=(dk, dv))
+    K = _unit(rng.normal(size=(n, dk)))
+    V = rng.normal(size=(n, dv))
+    beta = rng.uniform(0.1, 2.0)
+    alpha = rng.uniform(0.3, 1.0, size=dk)
+    S_tilde = alpha[:, None] * S_prev
+    Amat = np.vstack([np.eye(dk), np.sqrt(beta) * K])
+    rhs = np.vstack([S_tilde, np.sqrt(beta) * V])
+    want = np.linalg.lstsq(Amat, rhs, rcond=None)[0]
+    got = O.vda_update(S_prev, K, V, beta, alpha)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-10)
+    # and the gradient of the objective vanishes there
+    grad = (got - S_tilde) + beta * K.T @ (K @ got - V)
+    assert np.abs(grad).max() < 1e-10
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_orthonormal_keys_decouple(seed):
+    """With orthonormal keys (n <= d_k) the joint update equals independent
+    token-level delta rules with beta/(1+beta), applied in any order."""
+    rng = np.random.default_rng(200 + seed)
+    dk, dv, n = 8, 3, 5
+    Q, _ = np.linalg.qr(rng.normal(size=(dk, dk)))
+    K = Q[:, :n].T
+    V = rng.normal(size=(n, dv))
+    S = rng.normal(size=(dk, dv))
+    beta = rng.uniform(0.1, 2.0)
+    got = O.vda_update(S, K, V, beta)
+    for order in (range(n), reversed(range(n)), rng.permutation(n)):
+        want = S.copy()
+        for i in order:
+            want = _delta_rule_token(want, K[i], V[i], beta / (1 + beta))
+        np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-11)
+
+
+def test_beta_zero_is_pure_decay():
+    rng = np.random.default_rng(3)
+    S = rng.normal(size=(6, 6))
+    K = _unit(rng.normal(size=(9, 6)))
+    V = rng.normal(size=(9, 6))
+    alpha = rng.uniform(0, 1, size=6)
+    np.testing.assert_allclose(O.vda_update(S, K, V, 0.0, alpha), alpha[:, None] * S,
+                               rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_proposition1_non_expansive(seed):
+    """Proposition 1: for alpha in [0,1] and beta >= 0 the inherited-state map
+    is non-expansive in the spectral norm."""
+    rng = np.random.default_rng(300 + seed)
+    dk, dv, n = 10, 6, 30
+    K = rng.normal(size=(n, dk))
+    V = rng.normal(size=(n, dv))
+    beta = rng.uniform(0, 5)
+    alpha = rng.uniform(0, 1, size=dk)
+    for _ in range(20):
+        Sa = rng.normal(size=(dk, dv)) * rng.uniform(0.1, 10)
+        Sb = rng.normal(size=(dk, dv)) * rng.uniform(0.1, 10)
+        da = O.vda_update(Sa, K, V, beta, alpha) - O.vda_update(Sb, K, V, beta, alpha)
+        assert np.linalg.norm(da, 2) <= np.linalg.norm(Sa - Sb, 2) * (1 + 1e-12)
+
+
+def test_frozen_state_rule_differs_at_second_order():
+    """The frozen-state batched rule S = (I - A) S~ + W (all corrections at the
+    same decayed state) agrees with VDA to first order in beta; the gap
+    shrinks ~4x when beta halves.  A sign error in the key-space inverse would
+    make the gap first order (ratio ~2)."""
+    rng = np.random.default_rng(7)
+    dk, dv, n = 8, 5, 12
+    K = _unit(rng.normal(size=(n, dk)))
+    V = rng.normal(size=(n, dv))
+    S = rng.normal(size=(dk, dv))
+
+    def gap(beta):
+        A, W = beta * K.T @ K, beta * K.T @ V
+        frozen = (np.eye(dk) - A) @ S + W
+        return np.linalg.norm(O.vda_update(S, K, V, beta) - frozen)
+
+    r = gap(1e-3) / gap(5e-4)
+    assert 3.8 < r < 4.2
+
+
+# --- Regions, mask ------------------------------------------------------------
+
+def _brute_visible(tq, tk, T, C, r):
+    """Pairwise statement of the pages' rule: keys in a chunk at most r chunks
+    away, or the key frame is an anchor, or the query frame is an anchor."""
+    anchors = (0, T - 1)
+    near = abs(tq // C - tk // C) <= r
+    return near or tk in anchors or tq in anchors
+
+
+@pytest.mark.parametrize("T", list(range(1, 41)))
+def test_regions_disjoint_and_cover(T):
+    for C in range(1, 8):
+        for r in (1, 2):
+            M = O.frame_mask(T, C, r)
+            for tq in range(T):
+                S = set(O.softmax_key_frames(tq, T, C, r))
+                Fw = set(O.forward_region(tq, T, C, r))
+                Rv = set(O.reverse_region(tq, T, C, r))
+                assert not (S & Fw) and not (S & Rv) and not (Fw & Rv)
+                assert S | Fw | Rv == set(range(T))
+                assert all(f < min(S - {0, T - 1}, default=T) for f in Fw)
+                for tk in range(T):
+                    assert M[tq, tk] == _brute_visible(tq, tk, T, C, r)
+
+
+def test_token_mask_expands_frames():
+    T, N, C = 7, 3, 2
+    M = O.token_mask(T, N, C, 1)
+    for i, j in itertools.product(range(T * N), repeat=2):
+        assert M[i, j] == _brute_visible(i // N, j // N, T, C, 1)
+
+
+def test_window_is_15_frames_inside_clip():
+    """A query chunk away from the ends attends 3 chunks = 15 frames
+    ("producing a 15-frame window except at sequence boundaries")."""
+    T = 75
+    assert len(O.window_frames(37, T, 5, 1)) == 15
+    assert len(O.window_frames(2, T, 5, 1)) == 10       # shrunk at the start
+    assert len(O.window_frames(73, T, 5, 1)) == 10      # and at the end
+    # anchors counted once: chunk 0 already contains frame 0
+    assert O.softmax_key_frames(2, T, 5, 1) == list(range(10)) + [74]
+
+
+# --- Softmax branch -----------------------------------------------------------
+
+def test_softmax_bruteforce_tiny():
+    """Per-row enumeration with pure-Python loops over the visible keys."""
+    rng = np.random.default_rng(11)
+    B, T, N, H, d, C = 1, 7, 2, 2, 3, 2
+    L = T * N
+    q = rng.normal(size=(B, L, H, d)) * 2
+    k = rng.normal(size=(B, L, H, d))
+    v = rng.normal(size=(B, L, H, d))
+    got = O.softmax_branch(q, k, v, T, N, C, 1)
+    sc = 1 / np.sqrt(d)
+    for h in range(H):
+        for i in range(L):
+            vis = [j for j in range(L) if _brute_visible(i // N, j // N, T, C, 1)]
+            w = [np.exp(sc * sum(q[0, i, h, c] * k[0, j, h, c] for c in range(d))) for j in vis]
+            tot = sum(w)
+            want = [sum(w[a] * v[0, j, h, c] for a, j in enumerate(vis)) / tot for c in range(d)]
+            np.testing.assert_allclose(got[0, i, h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_window_spanning_clip_is_dense_softmax():
+    """One chunk covering the clip: the mask is full, so the Softmax branch is
+    dense attention (scipy.special.softmax)."""
+    rng = np.random.default_rng(12)
+    B, T, N, H, d = 2, 15, 4, 3, 8
+    L = T * N
+    q, k, v = (rng.normal(size=(B, L, H, d)) for _ in range(3))
+    got = O.softmax_branch(q, k, v, T, N, chunk=T, radius=1)
+    for b in range(B):
+        for h in range(H):
+            p = scipy.special.softmax(q[b, :, h] @ k[b, :, h].T / np.sqrt(d), axis=1)
+            np.testing.assert_allclose(got[b, :, h], p @ v[b, :, h], rtol=1e-11, atol=1e-12)
+
+
+# --- Linear branch --------------------------------------------------------------
+
+def _tiny_linear_inputs(seed, B=1, T=17, N=3, H=2, d=4, nt=5):
+    rng = np.random.default_rng(seed)
+    L = T * N
+    q = rng.normal(size=(B, L, H, d))
+    k = _unit(rng.normal(size=(B, L, H, d)))
+    v = rng.normal(size=(B, L, H, d))
+    tk = _unit(rng.normal(size=(B, nt, H, d)))
+    tv = rng.normal(size=(B, nt, H, d))
+    beta = scipy.special.expit(rng.normal(size=(B, H, 1 + T)))
+    alpha = rng.uniform(0.8, 1.0, size=(B, H, T, d))
+    return q, k, v, tk, tv, beta, alpha
+
+
+def test_text_counted_once():
+    """With every video write off (beta_1..T = 0) and alpha = 1, each query
+    reads exactly q^T S_text, whatever its frame (text counted once)."""
+    q, k, v, tk, tv, beta, _ = _tiny_linear_inputs(21)
+    T, N = 17, 3
+    beta[:, :, 1:] = 0
+    got = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1)
+    for h in range(2):
+        # S_text by least squares from the zero state
+        n = tk.shape[1]
+        Am = np.vstack([np.eye(4), np.sqrt(beta[0, h, 0]) * tk[0, :, h]])
+        rhs = np.vstack([np.zeros((4, 4)), np.sqrt(beta[0, h, 0]) * tv[0, :, h]])
+        S_text = np.linalg.lstsq(Am, rhs, rcond=None)[0]
+        assert n == 5
+        np.testing.assert_allclose(got[0, :, h], q[0, :, h] @ S_text, rtol=1e-11, atol=1e-12)
+
+
+def test_pure_decay_closed_form():
+    """No video writes, channel-wise decay: the forward readout carries
+    prod_{j<=t} alpha_j and the reverse one prod_{j>=t} alpha_j (every frame
+    between the text state and the query decays: frames outside the window,
+    anchors, and the bridge across the window).  Anchor queries: q^T S_text."""
+    q, k, v, tk, tv, beta, alpha = _tiny_linear_inputs(22)
+    T, N, d = 17, 3, 4
+    beta[:, :, 1:] = 0
+    got = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1, alpha=alpha)
+    for h in range(2):
+        St = O.text_state(tk[0, :, h], tv[0, :, h], beta[0, h, 0])
+        for i in range(T * N):
+            t = i // N
+            if t in (0, T - 1):
+                want = q[0, i, h] @ St
+            else:
+                gf = np.prod(alpha[0, h, :t + 1], axis=0)
+                gr = np.prod(alpha[0, h, t:], axis=0)
+                want = q[0, i, h] @ (0.5 * gf[:, None] * St) + q[0, i, h] @ (0.5 * gr[:, None] * St)
+            np.testing.assert_allclose(got[0, i, h], want, rtol=1e-11, atol=1e-12)
+
+
+def test_time_reversal_equivariance():
+    """Reversing the frame order (T a multiple of the chunk, so the chunk grid
+    and the window are symmetric) swaps the forward and reverse scans: the
+    linear readout of the reversed clip is the reversed readout."""
+    T, N, H, d = 20, 3, 2, 4
+    q, k, v, tk, tv, beta, alpha = _tiny_linear_inputs(23, T=T, N=N, H=H, d=d)
+
+    def rev_tok(x):
+        B, L = x.shape[:2]
+        return x.reshape(B, T, N, *x.shape[2:])[:, ::-1].reshape(x.shape)
+
+    beta_r = np.concatenate([beta[:, :, :1], beta[:, :, 1:][:, :, ::-1]], axis=2)
+    alpha_r = alpha[:, :, ::-1]
+    a = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1, alpha=alpha)
+    b = O.linear_branch(rev_tok(q), rev_tok(k), rev_tok(v), beta_r, tk, tv, T, N, 5, 1,
+                        alpha=alpha_r)
+    np.testing.assert_allclose(rev_tok(b), a, rtol=1e-10, atol=1e-11)
+
+
+def test_linear_regions_match_explicit_frame_sets():
+    """The readout equals q^T (forward state over exactly forward_region) +
+    q^T (reverse state over exactly reverse_region), built here by running the
+    delta-rule update over those explicit frame lists (alpha = 1)."""
+    T, N, H, d = 17, 3, 2, 4
+    q, k, v, tk, tv, beta, _ = _tiny_linear_inputs(24, T=T, N=N, H=H, d=d)
+    got = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1)
+    for h in range(H):
+        St = O.text_state(tk[0, :, h], tv[0, :, h], beta[0, h, 0])
+        for tq in range(T):
+            Sf = 0.5 * St
+            for t in O.forward_region(tq, T, 5, 1):
+                Sf = O.vda_update(Sf, k[0, t * N:(t + 1) * N, h], v[0, t * N:(t + 1) * N, h],
+                                  beta[0, h, 1 + t])
+            Sr = 0.5 * St
+            for t in reversed(O.reverse_region(tq, T, 5, 1)):
+                Sr = O.vda_update(Sr, k[0, t * N:(t + 1) * N, h], v[0, t * N:(t + 1) * N, h],
+                                  beta[0, h, 1 + t])
+            for n in range(N):
+                i = tq * N + n
+                np.testing.assert_allclose(got[0, i, h], q[0, i, h] @ Sf + q[0, i, h] @ Sr,
+                                           rtol=1e-11, atol=1e-12)
+
+
+def test_boundary_states_consistent_with_readout():
+    T, N, H, d = 17, 3, 2, 4
+    q, k, v, tk, tv, beta, _ = _tiny_linear_inputs(25, T=T, N=N, H=H, d=d)
+    F, G = O.boundary_states(k, v, beta, tk, tv, T, N, 5, 1)
+    got = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1)
+    for h in range(H):
+        for i in range(N, (T - 1) * N):
+            c = (i // N) // 5
+            np.testing.assert_allclose(got[0, i, h], q[0, i, h] @ (F[0, h, c] + G[0, h, c]),
+                                       rtol=1e-11, atol=1e-12)
+
+
+# --- Output -----------------------------------------------------------------------
+
+def test_rms_norm_properties():
+    rng = np.random.default_rng(31)
+    o = rng.normal(size=(2, 5, 3, 16)) * 3
+    y = O.rms_norm(o, eps=0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(O.rms_norm(7.5 * o, eps=0.0), y, rtol=1e-13)
+    ye = O.rms_norm(o, eps=1e-6)
+    ms = np.mean(o * o, axis=-1)
+    np.testing.assert_allclose(np.mean(ye * ye, axis=-1), ms / (ms + 1e-6), rtol=1e-12)
+
+
+def test_projection_head_blocks():
+    """Head h's gated branch outputs only reach the output through rows
+    h*d_v .. (h+1)*d_v of its own projection; zeroing a gate removes that
+    branch."""
+    rng = np.random.default_rng(32)
+    B, R, H, dv, Do = 1, 4, 3, 5, 7
+    os_, ol = rng.normal(size=(B, R, H, dv)), rng.normal(size=(B, R, H, dv))
+    gs, gl = rng.uniform(size=(B, R, H, dv)), rng.uniform(size=(B, R, H, dv))
+    Ws, Wl = rng.normal(size=(H * dv, Do)), rng.normal(size=(H * dv, Do))
+    full = O.output_projection(os_, ol, gs, gl, Ws, Wl)
+    no_lin = O.output_projection(os_, ol, gs, 0 * gl, Ws, Wl)
+    no_soft = O.output_projection(os_, ol, 0 * gs, gl, Ws, Wl)
+    np.testing.assert_allclose(full, no_lin + no_soft, rtol=1e-12, atol=1e-12)
+    Ws2 = Ws.copy()
+    Ws2[dv:2 * dv] = 0
+    os2 = os_.copy()
+    os2[:, :, 1] = 123.0
+    np.testing.assert_allclose(O.output_projection(os2, ol, gs, 0 * gl, Ws2, Wl),
+                               O.output_projection(os_, ol, gs, 0 * gl, Ws2, Wl), atol=1e-12)
+    # a single head, single channel: out = g * o * W[row]
+    one = O.output_projection(np.ones((1, 1, 1, 1)) * 2, np.zeros((1, 1, 1, 1)),
+                              np.full((1, 1, 1, 1), 0.5), np.zeros((1, 1, 1, 1)),
+                              np.array([[3.0, -1.0]]), np.zeros((1, 2)))
+    np.testing.assert_allclose(one, [[[3.0, -1.0]]])
