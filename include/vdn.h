@@ -38,20 +38,25 @@
  *   - Ownership: the caller owns every buffer (device memory unless stated).
  *     The library never allocates or frees device memory; all scratch comes
  *     from the caller's workspace (size from vdn_workspace_bytes).
- *   - Alignment: every pointer must be 16-byte aligned.
+ *   - Alignment: every pointer must be 16-byte aligned; the workspace 256-byte
+ *     aligned (any cudaMalloc / PyTorch allocation is).
  *   - Asynchrony: compute entry points validate arguments on the host, then
  *     enqueue kernels on `stream` and return without synchronising.  VDN_OK
  *     means "enqueued".  Device-side conditions (a bounded wait that expired,
  *     a value outside the range of an internal fp16 operand) are recorded in
- *     a status word inside the workspace; read it with vdn_device_status.
+ *     a status word inside the workspace, which every compute call clears when
+ *     it starts; read it with vdn_device_status after the call.
  *   - Errors: a failed validation returns before any launch and leaves every
  *     output untouched.  No exceptions cross the ABI.  The library keeps no
  *     global state except a per-device attribute cache; calls on different
  *     streams with different workspaces may run concurrently.
- *   - Supported: d_k == d_v in {32, 64, 128} (any d with VDN_FLAG_SIMT up to
- *     128), chunk >= 1, window_radius >= 0, T >= 1, N >= 1, n_text >= 0,
- *     D_out a multiple of 8.  Tensor-core kernels serve dtype BF16 with
- *     d in {64, 128}; every other case runs the exact-FP32 CUDA-core kernels.
+ *   - Supported: d_k == d_v in {32, 64, 128}, chunk >= 1, window_radius >= 0,
+ *     T >= 1, N >= 1, n_text >= 0, D_out a multiple of 8.  Tensor-core
+ *     kernels serve dtype BF16 with d in {64, 128} (Q K^T in bf16; P, V, the
+ *     gated branch outputs and W in fp16; FP32 accumulation, FP32 state);
+ *     every other case, and VDN_FLAG_SIMT, runs exact-FP32 CUDA-core kernels.
+ *   - Range (tensor-core path): |v|, |W_o_*| and |gate * branch output| must
+ *     stay below 65504 (fp16); an overflow sets VDN_ERR_RANGE.
  */
 #ifndef VDN_H_
 #define VDN_H_
@@ -64,6 +69,12 @@ extern "C" {
 #endif
 
 #define VDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define VDN_API __attribute__((visibility("default")))
+#else
+#define VDN_API
+#endif
 
 typedef enum vdn_status {
   VDN_OK = 0,
@@ -105,20 +116,20 @@ typedef struct vdn_params {
 } vdn_params;
 
 /* ABI version of the loaded library (VDN_ABI_VERSION). */
-int vdn_abi_version(void);
+VDN_API int vdn_abi_version(void);
 
 /* Static string for a status code; never NULL. */
-const char *vdn_status_string(vdn_status s);
+VDN_API const char *vdn_status_string(vdn_status s);
 
 /* Fills `p` with the pages' defaults for the given sizes: chunk 5,
  * window_radius 1, D_out = H*d, softmax_scale 0, rms_eps 1e-6, flags 0. */
-vdn_status vdn_params_init(vdn_params *p, int B, int H, int T, int N, int d,
+VDN_API vdn_status vdn_params_init(vdn_params *p, int B, int H, int T, int N, int d,
                            int n_text, vdn_dtype dtype);
 
 /* Workspace bytes needed by vdn_hybrid_attn_fwd, vdn_hybrid_attn_branches
  * and vdn_vda_boundary_states for these params (one size serves all three).
  * Host only; validates `p` like the compute calls. */
-vdn_status vdn_workspace_bytes(const vdn_params *p, size_t *bytes);
+VDN_API vdn_status vdn_workspace_bytes(const vdn_params *p, size_t *bytes);
 
 /* The whole hybrid attention forward:
  *   o_s = window+anchor Softmax(q, k, v)                          [B,L,H,d_v]
@@ -126,17 +137,38 @@ vdn_status vdn_workspace_bytes(const vdn_params *p, size_t *bytes);
  *   out = concat_h(g_s * o_s) W_o_soft + concat_h(g_l * RMS(o_l)) W_o_lin
  * alpha may be NULL (no decay).  n_text may be 0 (text_k/text_v may then be
  * NULL; S_text = 0).  Everything else is required. */
-vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const void *k,
+VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const void *k,
                                const void *v, const float *beta, const float *alpha,
                                const void *text_k, const void *text_v,
                                const void *W_o_soft, const void *W_o_lin,
                                const void *gates, void *out, void *workspace,
                                size_t workspace_bytes, vdn_stream_t stream);
 
+/* Stage boundaries recorded by vdn_hybrid_attn_fwd_staged. */
+#define VDN_STAGES 5 /* VDA states, operand conversion, Softmax, readout, projection */
+typedef struct vdn_stage_events {
+  void *events[VDN_STAGES + 1]; /* cudaEvent_t handles created by the caller */
+} vdn_stage_events;
+
+/* Same computation and arguments as vdn_hybrid_attn_fwd, and records
+ * events[0] before the first kernel and events[i] after stage i on `stream`:
+ * 1 VDA state path (frame statistics + solve, chunk composition, chunk scan),
+ * 2 operand conversion (V^T and W^T to fp16; empty on the CUDA-core path),
+ * 3 window+anchor Softmax, 4 linear readout (+ RMS norm and gate on the
+ * tensor-core path), 5 output projection.  Used for live per-stage timing
+ * with cudaEventElapsedTime.  `ev` may be NULL (no events). */
+VDN_API vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params *p, const void *q, const void *k,
+                                      const void *v, const float *beta, const float *alpha,
+                                      const void *text_k, const void *text_v,
+                                      const void *W_o_soft, const void *W_o_lin,
+                                      const void *gates, void *out, void *workspace,
+                                      size_t workspace_bytes, vdn_stream_t stream,
+                                      const vdn_stage_events *ev);
+
 /* The two branch readouts before gating and projection, float32
  * [B, L, H, d_v]: o_soft = Softmax branch, o_lin = linear branch before its
  * RMS norm.  Either output pointer may be NULL to skip that branch. */
-vdn_status vdn_hybrid_attn_branches(const vdn_params *p, const void *q, const void *k,
+VDN_API vdn_status vdn_hybrid_attn_branches(const vdn_params *p, const void *q, const void *k,
                                     const void *v, const float *beta, const float *alpha,
                                     const void *text_k, const void *text_v,
                                     float *o_soft, float *o_lin, void *workspace,
@@ -146,16 +178,16 @@ vdn_status vdn_hybrid_attn_branches(const vdn_params *p, const void *q, const vo
  * F[c] = forward state read by query chunk c (after every frame before its
  * window), G[c] = reverse state (after every frame after its window), before
  * the per-frame decay bridge.  Either output may be NULL. */
-vdn_status vdn_vda_boundary_states(const vdn_params *p, const void *k, const void *v,
+VDN_API vdn_status vdn_vda_boundary_states(const vdn_params *p, const void *k, const void *v,
                                    const float *beta, const float *alpha,
                                    const void *text_k, const void *text_v, float *F,
                                    float *G, void *workspace, size_t workspace_bytes,
                                    vdn_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
- * the last calls on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
- * VDN_ERR_RANGE).  `workspace` must be the one passed to those calls. */
-vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_stream_t stream);
+ * the last compute call on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
+ * VDN_ERR_RANGE).  `workspace` must be the one passed to that call. */
+VDN_API vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_stream_t stream);
 
 #ifdef __cplusplus
 }

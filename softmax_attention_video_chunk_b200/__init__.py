@@ -1,0 +1,260 @@
+"""softmax_attention_video_chunk_b200 -- Python binding of libvdn.
+
+Argument marshalling only: every step of the VDN hybrid attention forward
+runs in the CUDA kernels of ``libvdn.so`` (sm_100a), reached through its C ABI
+(``include/vdn.h``).  PyTorch supplies device memory and the stream.  There is
+no fallback: if the library is missing or the call fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvdn.so")
+
+VDN_F32, VDN_BF16 = 0, 1
+FLAG_TEXT_FULL, FLAG_SIMT = 1, 2
+
+STATUS = {
+    0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_SHAPE", 3: "VDN_ERR_DTYPE",
+    4: "VDN_ERR_ALIGNMENT", 5: "VDN_ERR_WORKSPACE", 6: "VDN_ERR_CUDA", 7: "VDN_ERR_TIMEOUT",
+    8: "VDN_ERR_UNSUPPORTED", 9: "VDN_ERR_RANGE",
+}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+
+class VdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({lib().vdn_status_string(code).decode()})")
+
+
+N_STAGES = 5
+STAGE_NAMES = ("vda_states", "convert", "softmax", "readout", "projection")
+
+
+class VdnStageEvents(ctypes.Structure):
+    _fields_ = [("events", ctypes.c_void_p * (N_STAGES + 1))]
+
+
+class VdnParams(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("N", ctypes.c_int),
+        ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("n_text", ctypes.c_int),
+        ("D_out", ctypes.c_int), ("chunk", ctypes.c_int), ("window_radius", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("softmax_scale", ctypes.c_float),
+        ("rms_eps", ctypes.c_float), ("flags", ctypes.c_uint),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvdn.so (built in-tree by ``__graft_entry__.build()`` or
+    ``python -m softmax_attention_video_chunk_b200._build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m softmax_attention_video_chunk_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        PP = ctypes.POINTER(VdnParams)
+        L.vdn_abi_version.restype = ctypes.c_int
+        L.vdn_status_string.restype = ctypes.c_char_p
+        L.vdn_status_string.argtypes = [ctypes.c_int]
+        L.vdn_params_init.restype = ctypes.c_int
+        L.vdn_params_init.argtypes = [PP] + [ctypes.c_int] * 7
+        L.vdn_workspace_bytes.restype = ctypes.c_int
+        L.vdn_workspace_bytes.argtypes = [PP, ctypes.POINTER(ctypes.c_size_t)]
+        L.vdn_hybrid_attn_fwd.restype = ctypes.c_int
+        L.vdn_hybrid_attn_fwd.argtypes = [PP] + [_P] * 12 + [ctypes.c_size_t, _P]
+        L.vdn_hybrid_attn_fwd_staged.restype = ctypes.c_int
+        L.vdn_hybrid_attn_fwd_staged.argtypes = ([PP] + [_P] * 12 + [ctypes.c_size_t, _P] +
+                                                 [ctypes.POINTER(VdnStageEvents)])
+        L.vdn_hybrid_attn_branches.restype = ctypes.c_int
+        L.vdn_hybrid_attn_branches.argtypes = [PP] + [_P] * 10 + [ctypes.c_size_t, _P]
+        L.vdn_vda_boundary_states.restype = ctypes.c_int
+        L.vdn_vda_boundary_states.argtypes = [PP] + [_P] * 9 + [ctypes.c_size_t, _P]
+        L.vdn_device_status.restype = ctypes.c_int
+        L.vdn_device_status.argtypes = [PP, _P, _P]
+        _lib = L
+    return _lib
+
+
+def make_params(B, H, T, N, d, n_text, dtype="bf16", *, chunk=5, window_radius=1,
+                D_out=None, out_dtype="f32", softmax_scale=0.0, rms_eps=1e-6,
+                text_full=False, simt=False) -> VdnParams:
+    p = VdnParams()
+    dt = {"f32": VDN_F32, "bf16": VDN_BF16}
+    rc = lib().vdn_params_init(ctypes.byref(p), B, H, T, N, d, n_text, dt[dtype])
+    p.chunk, p.window_radius = chunk, window_radius
+    p.D_out = H * d if D_out is None else D_out
+    p.out_dtype = dt[out_dtype]
+    p.softmax_scale, p.rms_eps = softmax_scale, rms_eps
+    p.flags = (FLAG_TEXT_FULL if text_full else 0) | (FLAG_SIMT if simt else 0)
+    size = ctypes.c_size_t(0)
+    rc = lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
+    if rc != 0:
+        raise VdnError(rc, "vdn_workspace_bytes")
+    return p
+
+
+def workspace_bytes(p: VdnParams) -> int:
+    size = ctypes.c_size_t(0)
+    rc = lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
+    if rc != 0:
+        raise VdnError(rc, "vdn_workspace_bytes")
+    return size.value
+
+
+# --------------------------------------------------------------------------
+# torch-facing wrappers (marshalling only)
+# --------------------------------------------------------------------------
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_name(t) -> str:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return "bf16"
+    if t.dtype == torch.float32:
+        return "f32"
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def params_for(q, v, text_k, T, W_soft=None, **kw) -> VdnParams:
+    B, L, H, d = q.shape
+    if L % T:
+        raise ValueError("q.shape[1] must be T * N")
+    n_text = 0 if text_k is None else text_k.shape[1]
+    D_out = None if W_soft is None else W_soft.shape[1]
+    return make_params(B, H, T, L // T, d, n_text, _dtype_name(q), D_out=D_out, **kw)
+
+
+def alloc_workspace(p: VdnParams, device="cuda"):
+    import torch
+    return torch.empty(max(workspace_bytes(p), 256), dtype=torch.uint8, device=device)
+
+
+def hybrid_attn_fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, *, alpha=None,
+                    out=None, workspace=None, stream=None, params=None, events=None, **kw):
+    """out [B, L, D_out] = VDN hybrid attention forward (all steps in libvdn).
+
+    ``events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
+    recorded at the stage boundaries (see vdn_hybrid_attn_fwd_staged)."""
+    import torch
+    p = params or params_for(q, v, text_k, T, W_soft, **kw)
+    if out is None:
+        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
+        out = torch.empty(q.shape[0], q.shape[1], p.D_out, dtype=odt, device=q.device)
+    ws = alloc_workspace(p, q.device) if workspace is None else workspace
+    ev = None
+    if events is not None:
+        if len(events) != N_STAGES + 1:
+            raise ValueError(f"need {N_STAGES + 1} events")
+        ev = VdnStageEvents()
+        for i, e in enumerate(events):
+            if not e.cuda_event:  # torch creates the CUDA event on first record
+                e.record(torch.cuda.current_stream() if stream is None else stream)
+            ev.events[i] = e.cuda_event
+        ev = ctypes.byref(ev)
+    rc = lib().vdn_hybrid_attn_fwd_staged(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                          _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(W_soft),
+                                          _ptr(W_lin), _ptr(gates), _ptr(out), _ptr(ws),
+                                          ws.numel(), _stream(stream), ev)
+    if rc != 0:
+        raise VdnError(rc, "vdn_hybrid_attn_fwd")
+    return out
+
+
+INPUT_NAMES = ("q", "k", "v", "beta", "alpha", "text_k", "text_v", "W_soft", "W_lin", "gates")
+
+
+def hybrid_attn_fwd_host(host: dict, T, *, device_bufs=None, out_host=None, workspace=None,
+                         stream=None, params=None, **kw):
+    """End-to-end call on host (pinned) tensors: copies every input to the
+    device, runs the forward, and copies ``out`` back into ``out_host``, all on
+    one stream.  ``device_bufs`` (same keys) are reused device buffers.
+    Returns (out_host, h2d_bytes, d2h_bytes)."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    s = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.stream(s):
+        if device_bufs is None:
+            device_bufs = {n: (None if host.get(n) is None else
+                               torch.empty_like(host[n], device=dev)) for n in INPUT_NAMES}
+        h2d = 0
+        for n in INPUT_NAMES:
+            if host.get(n) is not None:
+                device_bufs[n].copy_(host[n], non_blocking=True)
+                h2d += host[n].numel() * host[n].element_size()
+        d = device_bufs
+        out = hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                              d["W_soft"], d["W_lin"], d["gates"], T, alpha=d.get("alpha"),
+                              workspace=workspace, stream=s, params=params, **kw)
+        if out_host is None:
+            out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_host.copy_(out, non_blocking=True)
+    return out_host, h2d, out.numel() * out.element_size()
+
+
+def hybrid_attn_branches(q, k, v, beta, text_k, text_v, T, *, alpha=None, workspace=None,
+                         stream=None, want_soft=True, want_lin=True, params=None, **kw):
+    """(o_soft, o_lin) float32 [B, L, H, d]; o_lin before its RMS norm."""
+    import torch
+    p = params or params_for(q, v, text_k, T, **kw)
+    o_s = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_soft else None
+    o_l = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_lin else None
+    ws = alloc_workspace(p, q.device) if workspace is None else workspace
+    rc = lib().vdn_hybrid_attn_branches(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                        _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(o_s),
+                                        _ptr(o_l), _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_hybrid_attn_branches")
+    return o_s, o_l
+
+
+def vda_boundary_states(k, v, beta, text_k, text_v, T, *, alpha=None, workspace=None,
+                        stream=None, params=None, **kw):
+    """(F, G) float32 [B, H, n_chunks, d, d]: the forward / reverse state each
+    query chunk reads before its decay bridge."""
+    import torch
+    p = params or params_for(k, v, text_k, T, **kw)
+    nc = (p.T + p.chunk - 1) // p.chunk
+    F = torch.empty(p.B, p.H, nc, p.d_k, p.d_v, dtype=torch.float32, device=k.device)
+    G = torch.empty_like(F)
+    ws = alloc_workspace(p, k.device) if workspace is None else workspace
+    rc = lib().vdn_vda_boundary_states(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(beta),
+                                       _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(F),
+                                       _ptr(G), _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_vda_boundary_states")
+    return F, G
+
+
+def device_status(p: VdnParams, workspace, stream=None) -> int:
+    """Synchronise and return (and clear) the device status of the last call."""
+    return lib().vdn_device_status(ctypes.byref(p), _ptr(workspace), _stream(stream))
+
+
+def use_tc_params(p: VdnParams) -> bool:
+    """True when the call runs the tensor-core kernels (bf16, d in {64, 128})."""
+    return p.dtype == VDN_BF16 and p.d_k in (64, 128) and not (p.flags & FLAG_SIMT)

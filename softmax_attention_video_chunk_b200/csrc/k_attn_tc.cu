@@ -1,0 +1,439 @@
+// Window + anchor Softmax attention on the sm_100a tensor cores.
+//
+// "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
+// Generation", method, "Nearby frames ..." paragraph: exact Softmax over the
+// chunk-aligned window plus the two boundary anchors (four-way
+// connectivity), each key once.  The pages run this through a varlen
+// FlashAttention call with queries packed by visible-key pattern; here one
+// CTA owns two 128-row query tiles of one visible-key group (Geo::group) and
+// walks that group's key ranges directly.
+//
+// Per CTA (320 threads, one CTA per SM):
+//   warp 8      TMA producer: Q tiles once, then K (bf16) and V^T (fp16) tiles
+//               of 128 keys into a 2-stage ring;
+//   warp 9      MMA issuer (one thread): S_j = Q_j K^T (bf16, FP32 in TMEM),
+//               O_j += P_j V (P fp16 read from TMEM, V^T from smem);
+//   warps 0-3   softmax of query tile 0, warps 4-7 of tile 1: one thread per
+//               row reads its S row from TMEM, applies the key-range mask,
+//               keeps a running max (rescaling O in TMEM only when the max grows
+//               by more than 2^8) and row sum, writes P = 2^(s - m) as fp16
+//               over its S columns, and finally normalises O and writes
+//               g_s * o_s (fp16, the projection operand) or o_s (fp32).
+// TMEM (512 columns): S0 | S1 | O0 | O1.  Every mbarrier wait is bounded in
+// time; on expiry the CTA records VDN_ERR_TIMEOUT in the status word, drains
+// its MMAs and copies, frees TMEM and exits.
+#include <math.h>
+
+#include "tc_ptx.cuh"
+#include "vdn_common.cuh"
+#include "vdn_tc.h"
+
+namespace vdn {
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+struct Abort {
+  volatile int* flag;
+  int* status;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*ab.flag) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *ab.flag = 1;
+      atomicOr(ab.status, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+constexpr int kBK = 128;  // keys per tile
+
+// Key tile i of a group: tiles of each key range start at the range start
+// rounded down to 8 tokens (16-byte TMA coordinate of V^T); columns outside
+// [lo, hi) belong to no range of this group and are masked.
+__device__ __forceinline__ void kv_tile(const QGroup& g, int i, int& k0, int& lo, int& hi) {
+  k0 = 0; lo = 0; hi = 0;
+  for (int s = 0; s < g.nseg; ++s) {
+    const int a = g.seg0[s] & ~7;
+    const int nt = (g.seg1[s] - a + kBK - 1) / kBK;
+    if (i < nt) {
+      k0 = a + i * kBK;
+      lo = max(g.seg0[s], k0) - k0;
+      hi = min(g.seg1[s], k0 + kBK) - k0;
+      return;
+    }
+    i -= nt;
+  }
+}
+
+__device__ __forceinline__ int kv_count(const QGroup& g) {
+  int n = 0;
+  for (int s = 0; s < g.nseg; ++s) {
+    const int a = g.seg0[s] & ~7;
+    n += (g.seg1[s] - a + kBK - 1) / kBK;
+  }
+  return n;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+}  // namespace
+
+template <int D, bool FUSED>
+__global__ void __launch_bounds__(320, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+               const __grid_constant__ CUtensorMap map_vt, Geo geo, int B, int H,
+               float scale_log2, const __nv_bfloat16* __restrict__ gates,
+               __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status) {
+  constexpr int BM = 128, NS = 2;
+  constexpr int QT = BM * D * 2;   // bytes of a Q tile
+  constexpr int KT = kBK * D * 2;  // bytes of a K tile
+  constexpr int VT = kBK * D * 2;  // bytes of a V^T tile
+  constexpr int NSUB = D / 64;     // 128-byte column panels of a Q / K row
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 2 * QT;
+  uint8_t* sV = sK + NS * KT;
+  uint64_t* bars = (uint64_t*)(sV + NS * VT);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + NS;
+  uint64_t* kv_empty = v_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  int* abort_flag = (int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = B * H;
+  const int pair = blockIdx.x / BH, bh = blockIdx.x % BH;
+  const int b = bh / H, h = bh % H;
+  QGroup g;
+  int row0;
+  if (!find_tile(geo, 2 * BM, pair, &g, &row0)) return;  // uniform over the CTA
+  const int row_end = g.row0 + g.nrows;
+  const bool has1 = row0 + BM < row_end;
+  const int n_kv = kv_count(g);
+  const int L = geo.T * geo.N;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int i = 0; i < NS; ++i) {
+      ptx::mbar_init(k_full + i, 1);
+      ptx::mbar_init(v_full + i, 1);
+      ptx::mbar_init(kv_empty + i, 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      ptx::mbar_init(s_full + j, 1);
+      ptx::mbar_init(p_full + j, 128);
+      ptx::mbar_init(o_done + j, 1);
+    }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, status};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&map_q);
+      ptx::prefetch_tmap(&map_k);
+      ptx::prefetch_tmap(&map_vt);
+      ptx::mbar_arrive_expect_tx(q_full, (has1 ? 2 : 1) * QT);
+      for (int j = 0; j < (has1 ? 2 : 1); ++j)
+        for (int sub = 0; sub < NSUB; ++sub)
+          ptx::tma_load_4d(sQ + j * QT + sub * BM * 128, &map_q, q_full, sub * 64, h,
+                           row0 + j * BM, b);
+      int issued = 0;
+      for (int i = 0; i < n_kv; ++i) {
+        const int st = i % NS, use = i / NS;
+        if (use > 0 && !wait_bar(kv_empty + st, (use - 1) & 1, ab)) break;
+        int k0, lo, hi;
+        kv_tile(g, i, k0, lo, hi);
+        ptx::mbar_arrive_expect_tx(k_full + st, KT);
+        for (int sub = 0; sub < NSUB; ++sub)
+          ptx::tma_load_4d(sK + st * KT + sub * kBK * 128, &map_k, k_full + st, sub * 64, h, k0,
+                           b);
+        ptx::mbar_arrive_expect_tx(v_full + st, VT);
+        for (int vs = 0; vs < 2; ++vs)
+          ptx::tma_load_3d(sV + st * VT + vs * D * 128, &map_vt, v_full + st, k0 + vs * 64, 0,
+                           bh);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before the CTA releases its smem
+        const uint64_t t0 = ptx::globaltimer_ns();
+        for (int i = max(0, issued - NS); i < issued; ++i) {
+          const int st = i % NS, ph = (i / NS) & 1;
+          while (!ptx::mbar_try_wait(k_full + st, ph) && ptx::globaltimer_ns() - t0 < kWaitLimitNs) {}
+          while (!ptx::mbar_try_wait(v_full + st, ph) && ptx::globaltimer_ns() - t0 < kWaitLimitNs) {}
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = ptx::idesc_f16(128, kBK, 1);
+      constexpr uint32_t idO = ptx::idesc_f16(128, D, 0);
+      const uint32_t sQa = ptx::smem_u32(sQ), sKa = ptx::smem_u32(sK), sVa = ptx::smem_u32(sV);
+      auto issue_S = [&](int j, int st) {
+        const uint32_t d = tmem + j * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint64_t a = ptx::sdesc_k_sw128(sQa + j * QT + off);
+          const uint64_t bd = ptx::sdesc_k_sw128(sKa + st * KT + (kk >> 2) * (kBK * 128) + (kk & 3) * 32);
+          ptx::mma_ss(d, a, bd, idS, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(s_full + j);
+      };
+      auto issue_PV = [&](int j, int st, bool first) {
+        const uint32_t d = tmem + 256 + j * D;
+        const uint32_t pa = tmem + j * 128;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t bd = ptx::sdesc_k_sw128(sVa + st * VT + (kk >> 2) * (D * 128) + (kk & 3) * 32);
+          ptx::mma_ts(d, pa + kk * 8, bd, idO, (!first || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(o_done + j);
+      };
+      bool ok = wait_bar(q_full, 0, ab) && wait_bar(k_full, 0, ab);
+      if (ok) {
+        ptx::tc_fence_after();
+        issue_S(0, 0);
+        if (has1) issue_S(1, 0);
+      }
+      for (int i = 0; ok && i < n_kv; ++i) {
+        const int st = i % NS, ph = (i / NS) & 1;
+        const int st2 = (i + 1) % NS, ph2 = ((i + 1) / NS) & 1;
+        if (!(ok = wait_bar(v_full + st, ph, ab))) break;
+        if (!(ok = wait_bar(p_full + 0, i & 1, ab))) break;
+        ptx::tc_fence_after();
+        issue_PV(0, st, i == 0);
+        if (i + 1 < n_kv) {
+          if (!(ok = wait_bar(k_full + st2, ph2, ab))) break;
+          ptx::tc_fence_after();
+          issue_S(0, st2);
+        }
+        if (has1) {
+          if (!(ok = wait_bar(p_full + 1, i & 1, ab))) break;
+          ptx::tc_fence_after();
+          issue_PV(1, st, i == 0);
+        }
+        ptx::mma_commit(kv_empty + st);
+        if (has1 && i + 1 < n_kv) issue_S(1, st2);
+      }
+      // every MMA of this CTA completes before TMEM is released
+      ptx::mma_commit(drain);
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!ptx::mbar_try_wait(drain, 0) && ptx::globaltimer_ns() - t0 < kWaitLimitNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int j = warp >> 2, wq = warp & 3;
+    if (j == 0 || has1) {
+      const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_off + j * 128;
+      const uint32_t tO = tmem + lane_off + 256 + j * D;
+      float m_used = -INFINITY, l_sum = 0.f;
+      bool ok = true;
+      for (int i = 0; i < n_kv; ++i) {
+        int k0, lo, hi;
+        kv_tile(g, i, k0, lo, hi);
+        if (!(ok = wait_bar(s_full + j, i & 1, ab))) break;
+        ptx::tc_fence_after();
+        // pass 1: row maximum over the valid key columns (log2 domain)
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS + 32 * c, r);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = 32 * c + e;
+            if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(r[e]) * scale_log2);
+          }
+        }
+        if (i == 0) {
+          m_used = mx;
+        } else {
+          const bool need = mx > m_used + 8.f;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = fmaxf(m_used, mx);
+            const float f = ptx::ex2(m_used - m_new);
+            l_sum *= f;
+            m_used = m_new;
+            if (!(ok = wait_bar(o_done + j, (i - 1) & 1, ab))) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              ptx::tmem_ld32(tO + 32 * c, o);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              ptx::tmem_st32(tO + 32 * c, o);
+            }
+            ptx::tmem_wait_st();
+          }
+        }
+        // pass 2: P = 2^(s - m) as fp16 pairs over the first 64 columns of S
+        float sum = 0.f;
+        const float neg_m = -m_used;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ra[32], rb[32], pk[32];
+          ptx::tmem_ld32(tS + 64 * half, ra);
+          ptx::tmem_ld32(tS + 64 * half + 32, rb);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 64 * half + 2 * e;
+            float p0 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e]), scale_log2, neg_m));
+            float p1 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e + 1]), scale_log2, neg_m));
+            p0 = (c0 >= lo && c0 < hi) ? p0 : 0.f;
+            p1 = (c0 + 1 >= lo && c0 + 1 < hi) ? p1 : 0.f;
+            sum += p0 + p1;
+            pk[e] = pack_half2(p0, p1);
+            const int c1 = c0 + 32;
+            float q0 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e]), scale_log2, neg_m));
+            float q1 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e + 1]), scale_log2, neg_m));
+            q0 = (c1 >= lo && c1 < hi) ? q0 : 0.f;
+            q1 = (c1 + 1 >= lo && c1 + 1 < hi) ? q1 : 0.f;
+            sum += q0 + q1;
+            pk[16 + e] = pack_half2(q0, q1);
+          }
+          ptx::tmem_st32(tS + 32 * half, pk);
+        }
+        ptx::tmem_wait_st();
+        l_sum += sum;
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(p_full + j);
+      }
+      if (ok && n_kv > 0 && wait_bar(o_done + j, (n_kv - 1) & 1, ab)) {
+        ptx::tc_fence_after();
+        const int row = row0 + j * BM + wq * 32 + lane;
+        const bool valid = row < row_end;
+        const float inv = 1.f / l_sum;
+        const size_t tok = (size_t)b * L + row;
+        bool bad = false;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + 32 * c, o);
+          ptx::tmem_wait_ld();
+          if (!valid) continue;
+          if constexpr (FUSED) {
+            const uint4* gp = reinterpret_cast<const uint4*>(gates + (tok * H + h) * D + 32 * c);
+            uint4* xp = reinterpret_cast<uint4*>(x + tok * (size_t)(2 * H * D) + (size_t)h * D + 32 * c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const uint4 gg = gp[v4];
+              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gg);
+              uint4 outv;
+              uint32_t* ow = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 gf = __bfloat1622float2(g2[e]);
+                const float a0 = gf.x * __uint_as_float(o[8 * v4 + 2 * e]) * inv;
+                const float a1 = gf.y * __uint_as_float(o[8 * v4 + 2 * e + 1]) * inv;
+                bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
+                ow[e] = pack_half2(a0, a1);
+              }
+              xp[v4] = outv;
+            }
+          } else {
+            float4* op = reinterpret_cast<float4*>(o_s + (tok * H + h) * D + 32 * c);
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              op[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv, __uint_as_float(o[4 * v4 + 1]) * inv,
+                                   __uint_as_float(o[4 * v4 + 2]) * inv, __uint_as_float(o[4 * v4 + 3]) * inv);
+          }
+        }
+        if (bad) atomicOr(status, kDevRange);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
+
+template <int D, bool FUSED>
+static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float* o_s,
+                                 cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const uint64_t L = t.L, H = t.H, B = t.B;
+  {
+    const uint64_t dims[4] = {(uint64_t)D, H, L, B};
+    const uint64_t str[3] = {(uint64_t)D * 2, H * D * 2, L * H * D * 2};
+    const uint32_t box[4] = {64, 1, 128, 1};
+    if (!make_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.q, dims, str, box))
+      return cudaErrorInvalidValue;
+    if (!make_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.k, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)t.Lp, (uint64_t)D, B * H};
+    const uint64_t str[2] = {(uint64_t)t.Lp * 2, (uint64_t)D * t.Lp * 2};
+    const uint32_t box[3] = {64, (uint32_t)D, 1};
+    if (!make_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, t.vt, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  Geo geo{t.T, t.N, t.C, t.R};
+  const int pairs = count_tiles(geo, 256);
+  const size_t sm = 1024 + 2 * (128 * D * 2) + 2 * 2 * (128 * D * 2) + 256;
+  auto kern = attn_tc_kernel<D, FUSED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const float scale_log2 = t.scale * 1.4426950408889634f;
+  const unsigned grid = (unsigned)pairs * (unsigned)(t.B * t.H);
+  kern<<<grid, 320, sm, st>>>(mq, mk, mv, geo, t.B, t.H, scale_log2,
+                              FUSED ? (const __nv_bfloat16*)f->gates : nullptr,
+                              FUSED ? f->x : nullptr, o_s, t.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc(const TcAttnArgs& t, const TcFwdArgs* f, float* o_s, cudaStream_t st) {
+  if (f != nullptr) {
+    if (t.D == 128) return launch_attn_t<128, true>(t, f, nullptr, st);
+    if (t.D == 64) return launch_attn_t<64, true>(t, f, nullptr, st);
+  } else {
+    if (t.D == 128) return launch_attn_t<128, false>(t, nullptr, o_s, st);
+    if (t.D == 64) return launch_attn_t<64, false>(t, nullptr, o_s, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

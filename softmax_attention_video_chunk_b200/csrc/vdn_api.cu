@@ -1,0 +1,322 @@
+// C ABI of libvdn: argument validation, workspace layout, launch sequence.
+//
+// The call sequence follows the pages' forward (method section of "Video
+// DeltaNet: A Video-Native Hybrid Attention for Livestream Video
+// Generation"): the VDA state path (frame statistics -> Gauss-Jordan solve ->
+// chunk composition -> bidirectional chunk scan), the window+anchor Softmax,
+// the linear readout with its decay bridge, then the gated dual output
+// projection.  Every step runs in this library's kernels; PyTorch (or any
+// caller) only provides device memory and the stream.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "vdn_common.cuh"
+#include "vdn_kernels.h"
+#include "vdn_tc.h"
+
+namespace vdn {
+
+static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t status, Mf, Rf, CM, CR, FS, GS;   // VDA state path
+  size_t o_s, o_l, rinv;                   // CUDA-core path intermediates
+  size_t vt, wt, x;                        // tensor-core path operands
+  size_t total;
+};
+
+static WsLayout layout(const vdn_params& p) {
+  WsLayout w;
+  memset(&w, 0, sizeof(w));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t B = p.B, H = p.H, T = p.T, d = p.d_k;
+  const size_t L = (size_t)p.T * p.N;
+  const size_t nc = (p.T + p.chunk - 1) / p.chunk;
+  const size_t mat = d * d * sizeof(float);
+  w.status = take(256);
+  w.Mf = take(B * H * (T + 1) * mat);
+  w.Rf = take(B * H * (T + 1) * mat);
+  w.CM = take(2 * B * H * nc * mat);
+  w.CR = take(2 * B * H * nc * mat);
+  w.FS = take(B * H * (nc + 1) * mat);
+  w.GS = take(B * H * (nc + 1) * mat);
+  if (use_tc(p)) {
+    TcSizes s = tc_sizes(p);
+    w.vt = take(s.vt_bytes);
+    w.wt = take(s.wt_bytes);
+    w.x = take(s.x_bytes);
+  } else {
+    w.o_s = take(B * L * H * d * sizeof(float));
+    w.o_l = take(B * L * H * d * sizeof(float));
+    w.rinv = take(B * L * H * sizeof(float));
+  }
+  w.total = off;
+  return w;
+}
+
+static vdn_status validate_params(const vdn_params* p) {
+  if (p == nullptr) return VDN_ERR_INVALID_ARG;
+  if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT)) return VDN_ERR_INVALID_ARG;
+  if ((p->dtype != VDN_F32 && p->dtype != VDN_BF16) ||
+      (p->out_dtype != VDN_F32 && p->out_dtype != VDN_BF16))
+    return VDN_ERR_DTYPE;
+  if (p->B < 1 || p->H < 1 || p->T < 1 || p->N < 1 || p->n_text < 0 || p->chunk < 1 ||
+      p->window_radius < 0 || p->D_out < 1)
+    return VDN_ERR_SHAPE;
+  if (p->d_k != p->d_v) return VDN_ERR_UNSUPPORTED;
+  if (p->d_k != 32 && p->d_k != 64 && p->d_k != 128) return VDN_ERR_UNSUPPORTED;
+  if (p->D_out % 8 != 0) return VDN_ERR_SHAPE;
+  if (!(p->softmax_scale >= 0.f) || isinf(p->softmax_scale)) return VDN_ERR_INVALID_ARG;
+  if (!(p->rms_eps >= 0.f) || isinf(p->rms_eps)) return VDN_ERR_INVALID_ARG;
+  // index ranges: tokens and grid sizes
+  const double L = (double)p->T * p->N;
+  if (L > 2147483647.0 / 2) return VDN_ERR_SHAPE;
+  if ((double)p->B * L * p->H * p->d_k > 9.0e15) return VDN_ERR_SHAPE;
+  if (p->H > 65535 || p->B > 32767 || p->T + 1 > 2147483647 / 2) return VDN_ERR_SHAPE;
+  return VDN_OK;
+}
+
+static inline bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+static vdn_status check_ptr(const void* ptr, bool required) {
+  if (ptr == nullptr) return required ? VDN_ERR_INVALID_ARG : VDN_OK;
+  return aligned16(ptr) ? VDN_OK : VDN_ERR_ALIGNMENT;
+}
+
+static vdn_status check_ws(const vdn_params* p, const void* ws, size_t ws_bytes) {
+  const WsLayout w = layout(*p);
+  if (ws == nullptr || ws_bytes < w.total) return VDN_ERR_WORKSPACE;
+  if (((uintptr_t)ws & 255u) != 0) return VDN_ERR_ALIGNMENT;
+  return VDN_OK;
+}
+
+#define VDN_TRY(expr)                        \
+  do {                                       \
+    vdn_status _s = (expr);                  \
+    if (_s != VDN_OK) return _s;             \
+  } while (0)
+
+#define VDN_CUDA(expr)                                   \
+  do {                                                   \
+    if ((expr) != cudaSuccess) return VDN_ERR_CUDA;      \
+  } while (0)
+
+static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const float* beta,
+                        const float* alpha, const void* text_k, const void* text_v, char* ws) {
+  const WsLayout w = layout(*p);
+  VdaArgs a;
+  a.B = p->B; a.H = p->H; a.T = p->T; a.N = p->N; a.D = p->d_k; a.C = p->chunk;
+  a.R = p->window_radius; a.n_text = p->n_text; a.dtype = p->dtype;
+  a.init_scale = (p->flags & VDN_FLAG_TEXT_FULL) ? 1.f : 0.5f;
+  a.k = k; a.v = v; a.text_k = text_k; a.text_v = text_v; a.beta = beta; a.alpha = alpha;
+  a.Mf = (float*)(ws + w.Mf); a.Rf = (float*)(ws + w.Rf);
+  a.CM = (float*)(ws + w.CM); a.CR = (float*)(ws + w.CR);
+  a.FS = (float*)(ws + w.FS); a.GS = (float*)(ws + w.GS);
+  return a;
+}
+
+static AttnArgs attn_args(const vdn_params* p, const void* q, const void* k, const void* v) {
+  AttnArgs a;
+  a.B = p->B; a.H = p->H; a.T = p->T; a.N = p->N; a.D = p->d_k; a.C = p->chunk;
+  a.R = p->window_radius; a.dtype = p->dtype;
+  a.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.f / sqrtf((float)p->d_k);
+  a.q = q; a.k = k; a.v = v;
+  return a;
+}
+
+static vdn_status common_inputs(const vdn_params* p, const void* q, const void* k, const void* v,
+                                const float* beta, const float* alpha, const void* text_k,
+                                const void* text_v, bool need_q) {
+  VDN_TRY(check_ptr(q, need_q));
+  VDN_TRY(check_ptr(k, true));
+  VDN_TRY(check_ptr(v, true));
+  VDN_TRY(check_ptr(beta, true));
+  VDN_TRY(check_ptr(alpha, false));
+  VDN_TRY(check_ptr(text_k, p->n_text > 0));
+  VDN_TRY(check_ptr(text_v, p->n_text > 0));
+  return VDN_OK;
+}
+
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+int vdn_abi_version(void) { return VDN_ABI_VERSION; }
+
+const char* vdn_status_string(vdn_status s) {
+  switch (s) {
+    case VDN_OK: return "VDN_OK";
+    case VDN_ERR_INVALID_ARG: return "VDN_ERR_INVALID_ARG: missing pointer or invalid flag/value";
+    case VDN_ERR_SHAPE: return "VDN_ERR_SHAPE: size out of range";
+    case VDN_ERR_DTYPE: return "VDN_ERR_DTYPE: unsupported dtype";
+    case VDN_ERR_ALIGNMENT: return "VDN_ERR_ALIGNMENT: pointer not 16-byte aligned (workspace: 256)";
+    case VDN_ERR_WORKSPACE: return "VDN_ERR_WORKSPACE: workspace missing or too small";
+    case VDN_ERR_CUDA: return "VDN_ERR_CUDA: CUDA runtime error";
+    case VDN_ERR_TIMEOUT: return "VDN_ERR_TIMEOUT: bounded device wait expired";
+    case VDN_ERR_UNSUPPORTED: return "VDN_ERR_UNSUPPORTED: configuration not served";
+    case VDN_ERR_RANGE: return "VDN_ERR_RANGE: value outside the range of an fp16 operand";
+  }
+  return "VDN_ERR_UNKNOWN";
+}
+
+vdn_status vdn_params_init(vdn_params* p, int B, int H, int T, int N, int d, int n_text,
+                           vdn_dtype dtype) {
+  if (p == nullptr) return VDN_ERR_INVALID_ARG;
+  memset(p, 0, sizeof(*p));
+  p->B = B; p->H = H; p->T = T; p->N = N; p->d_k = d; p->d_v = d; p->n_text = n_text;
+  p->D_out = H * d; p->chunk = 5; p->window_radius = 1; p->dtype = dtype;
+  p->out_dtype = VDN_F32; p->softmax_scale = 0.f; p->rms_eps = 1e-6f; p->flags = 0;
+  return validate_params(p);
+}
+
+vdn_status vdn_workspace_bytes(const vdn_params* p, size_t* bytes) {
+  if (bytes == nullptr) return VDN_ERR_INVALID_ARG;
+  VDN_TRY(validate_params(p));
+  *bytes = layout(*p).total;
+  return VDN_OK;
+}
+
+vdn_status vdn_vda_boundary_states(const vdn_params* p, const void* k, const void* v,
+                                   const float* beta, const float* alpha, const void* text_k,
+                                   const void* text_v, float* F, float* G, void* workspace,
+                                   size_t workspace_bytes, vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  VDN_TRY(common_inputs(p, nullptr, k, v, beta, alpha, text_k, text_v, false));
+  VDN_TRY(check_ptr(F, false));
+  VDN_TRY(check_ptr(G, false));
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  VdaArgs a = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+  VDN_CUDA(launch_vda_states(a, st));
+  if (F != nullptr || G != nullptr) VDN_CUDA(launch_gather_boundary(a, F, G, st));
+  return VDN_OK;
+}
+
+vdn_status vdn_hybrid_attn_branches(const vdn_params* p, const void* q, const void* k,
+                                    const void* v, const float* beta, const float* alpha,
+                                    const void* text_k, const void* text_v, float* o_soft,
+                                    float* o_lin, void* workspace, size_t workspace_bytes,
+                                    vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  VDN_TRY(common_inputs(p, q, k, v, beta, alpha, text_k, text_v, true));
+  VDN_TRY(check_ptr(o_soft, false));
+  VDN_TRY(check_ptr(o_lin, false));
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  const WsLayout w = layout(*p);
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  const bool tc = use_tc(*p);
+  if (o_lin != nullptr) {
+    VdaArgs a = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+    VDN_CUDA(launch_vda_states(a, st));
+    VDN_CUDA(launch_vda_readout_simt(a, q, o_lin, st));
+  }
+  if (o_soft != nullptr) {
+    AttnArgs a = attn_args(p, q, k, v);
+    if (tc) {
+      TcAttnArgs t = tc_attn_args(*p, a, ws + w.vt, (int*)(ws + w.status));
+      VDN_CUDA(launch_convert_v(t, st));
+      VDN_CUDA(launch_attn_tc(t, nullptr, o_soft, st));
+    } else {
+      VDN_CUDA(launch_attn_simt(a, o_soft, st));
+    }
+  }
+  return VDN_OK;
+}
+
+vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const void* k,
+                                      const void* v, const float* beta, const float* alpha,
+                                      const void* text_k, const void* text_v,
+                                      const void* W_o_soft, const void* W_o_lin,
+                                      const void* gates, void* out, void* workspace,
+                                      size_t workspace_bytes, vdn_stream_t stream,
+                                      const vdn_stage_events* ev) {
+  VDN_TRY(validate_params(p));
+  VDN_TRY(common_inputs(p, q, k, v, beta, alpha, text_k, text_v, true));
+  VDN_TRY(check_ptr(W_o_soft, true));
+  VDN_TRY(check_ptr(W_o_lin, true));
+  VDN_TRY(check_ptr(gates, true));
+  VDN_TRY(check_ptr(out, true));
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  if (ev != nullptr)
+    for (int i = 0; i <= VDN_STAGES; ++i)
+      if (ev->events[i] == nullptr) return VDN_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  auto mark = [&](int i) -> cudaError_t {
+    return ev ? cudaEventRecord((cudaEvent_t)ev->events[i], st) : cudaSuccess;
+  };
+  char* ws = (char*)workspace;
+  const WsLayout w = layout(*p);
+  VDN_CUDA(mark(0));
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  VdaArgs va = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+  AttnArgs aa = attn_args(p, q, k, v);
+  if (use_tc(*p)) {
+    TcAttnArgs t = tc_attn_args(*p, aa, ws + w.vt, (int*)(ws + w.status));
+    TcFwdArgs f = tc_fwd_args(*p, va, t, W_o_soft, W_o_lin, gates, out, ws + w.wt, ws + w.x);
+    VDN_CUDA(launch_vda_states(va, st));
+    VDN_CUDA(mark(1));
+    VDN_CUDA(launch_convert_v(t, st));
+    VDN_CUDA(launch_convert_w(f, st));
+    VDN_CUDA(mark(2));
+    VDN_CUDA(launch_attn_tc(t, &f, nullptr, st));
+    VDN_CUDA(mark(3));
+    VDN_CUDA(launch_readout_tc(f, st));
+    VDN_CUDA(mark(4));
+    VDN_CUDA(launch_gemm_tc(f, st));
+    VDN_CUDA(mark(5));
+    return VDN_OK;
+  }
+  float* o_s = (float*)(ws + w.o_s);
+  float* o_l = (float*)(ws + w.o_l);
+  VDN_CUDA(launch_vda_states(va, st));
+  VDN_CUDA(mark(1));
+  VDN_CUDA(mark(2));
+  VDN_CUDA(launch_attn_simt(aa, o_s, st));
+  VDN_CUDA(mark(3));
+  VDN_CUDA(launch_vda_readout_simt(va, q, o_l, st));
+  VDN_CUDA(mark(4));
+  ProjArgs pa;
+  pa.B = p->B; pa.H = p->H; pa.L = p->T * p->N; pa.D = p->d_k; pa.D_out = p->D_out;
+  pa.dtype = p->dtype; pa.out_dtype = p->out_dtype; pa.eps = p->rms_eps;
+  pa.o_s = o_s; pa.o_l = o_l; pa.gates = gates; pa.W_soft = W_o_soft; pa.W_lin = W_o_lin;
+  pa.rinv = (float*)(ws + w.rinv); pa.out = out;
+  VDN_CUDA(launch_proj_simt(pa, st));
+  VDN_CUDA(mark(5));
+  return VDN_OK;
+}
+
+vdn_status vdn_hybrid_attn_fwd(const vdn_params* p, const void* q, const void* k, const void* v,
+                               const float* beta, const float* alpha, const void* text_k,
+                               const void* text_v, const void* W_o_soft, const void* W_o_lin,
+                               const void* gates, void* out, void* workspace,
+                               size_t workspace_bytes, vdn_stream_t stream) {
+  return vdn_hybrid_attn_fwd_staged(p, q, k, v, beta, alpha, text_k, text_v, W_o_soft, W_o_lin,
+                                    gates, out, workspace, workspace_bytes, stream, nullptr);
+}
+
+vdn_status vdn_device_status(const vdn_params* p, void* workspace, vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  if (workspace == nullptr) return VDN_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaStreamSynchronize(st));
+  int word = 0;
+  VDN_CUDA(cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost));
+  VDN_CUDA(cudaMemset(workspace, 0, sizeof(int)));
+  if (word & kDevTimeout) return VDN_ERR_TIMEOUT;
+  if (word & kDevRange) return VDN_ERR_RANGE;
+  return VDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal launch interface between the C ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/vdn.h"
+
+namespace vdn {
+
+struct VdaArgs {
+  int B, H, T, N, D, C, R, n_text;
+  vdn_dtype dtype;
+  float init_scale;  // 0.5 (text counted once over the two scans) or 1
+  const void *k, *v, *text_k, *text_v;
+  const float *beta, *alpha;
+  // workspace: per-frame transitions [B][H][T+1][D][D]; chunk maps
+  // [2][B][H][nc][D][D]; boundary states [B][H][nc+1][D][D]
+  float *Mf, *Rf, *CM, *CR, *FS, *GS;
+};
+
+cudaError_t launch_vda_states(const VdaArgs& a, cudaStream_t st);
+cudaError_t launch_vda_readout_simt(const VdaArgs& a, const void* q, float* o_l, cudaStream_t st);
+cudaError_t launch_gather_boundary(const VdaArgs& a, float* F, float* G, cudaStream_t st);
+
+struct AttnArgs {
+  int B, H, T, N, D, C, R;
+  vdn_dtype dtype;
+  float scale;
+  const void *q, *k, *v;
+};
+cudaError_t launch_attn_simt(const AttnArgs& a, float* o_s, cudaStream_t st);
+
+struct ProjArgs {
+  int B, H, L, D, D_out;
+  vdn_dtype dtype, out_dtype;
+  float eps;
+  const float *o_s, *o_l;  // [B*L, H*D] fp32
+  const void *gates;       // [2][B*L][H*D]
+  const void *W_soft, *W_lin;  // [H*D][D_out]
+  float* rinv;             // [B*L*H] scratch
+  void* out;
+};
+cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t st);
+
+}  // namespace vdn

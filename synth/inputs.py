@@ -126,17 +126,19 @@ def make_inputs(cfg: Config, *, alpha_range: Optional[tuple] = None,
 
 
 def sample_rows(cfg: Config, per_frame: int = 4, extra_frac: float = 0.0,
-                seed: int = 12345) -> np.ndarray:
+                seed: int = 12345, chunks=None) -> np.ndarray:
     """Seeded sample of query token indices (within one batch item).
 
     Takes ``per_frame`` tokens (the first, the last and random ones) from:
     frames 0 and T-1 (the anchors) and the first and last frame of every
-    chunk, plus a random ``extra_frac`` of all other tokens.  Sorted, unique.
+    chunk (or of the chunks listed in ``chunks``), plus a random
+    ``extra_frac`` of all other tokens.  Sorted, unique.
     """
     rng = np.random.default_rng(seed)
     T, N, C = cfg.T, cfg.N, cfg.chunk
     frames = {0, T - 1}
-    for c in range((T + C - 1) // C):
+    nc = (T + C - 1) // C
+    for c in (range(nc) if chunks is None else [c % nc for c in chunks]):
         frames.add(c * C)
         frames.add(min(T, (c + 1) * C) - 1)
     rows = []

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, and validates its arguments before any
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import softmax_attention_video_chunk_b200 as vdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_lib():
+    from softmax_attention_video_chunk_b200 import _build
+    if _build.needs_build():
+        _build.build()
+    return vdn.lib()
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "vdn.h")).read()
+    return re.findall(r"VDN_API[^;{]*?\b(vdn_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol():
+    syms = _declared_symbols()
+    assert len(syms) >= 8
+    L = vdn.lib()
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+def test_abi_version_and_strings():
+    L = vdn.lib()
+    assert L.vdn_abi_version() == 1
+    for code in range(10):
+        assert L.vdn_status_string(code)
+    assert b"UNKNOWN" in L.vdn_status_string(99)
+
+
+def test_params_init_defaults():
+    p = vdn.VdnParams()
+    assert vdn.lib().vdn_params_init(ctypes.byref(p), 1, 24, 75, 1536, 128, 512, vdn.VDN_BF16) == 0
+    assert (p.chunk, p.window_radius, p.D_out, p.out_dtype) == (5, 1, 24 * 128, vdn.VDN_F32)
+    assert abs(p.rms_eps - 1e-6) < 1e-12 and p.softmax_scale == 0.0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("B", 0, "VDN_ERR_SHAPE"), ("T", 0, "VDN_ERR_SHAPE"), ("N", 0, "VDN_ERR_SHAPE"),
+    ("chunk", 0, "VDN_ERR_SHAPE"), ("window_radius", -1, "VDN_ERR_SHAPE"),
+    ("n_text", -1, "VDN_ERR_SHAPE"), ("D_out", 12, "VDN_ERR_SHAPE"),
+    ("d_v", 32, "VDN_ERR_UNSUPPORTED"), ("dtype", 7, "VDN_ERR_DTYPE"),
+    ("out_dtype", 3, "VDN_ERR_DTYPE"), ("flags", 1 << 5, "VDN_ERR_INVALID_ARG"),
+    ("softmax_scale", -1.0, "VDN_ERR_INVALID_ARG"), ("rms_eps", float("nan"), "VDN_ERR_INVALID_ARG"),
+])
+def test_param_validation(field, value, code):
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    setattr(p, field, value)
+    size = ctypes.c_size_t(0)
+    rc = vdn.lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
+    assert vdn.STATUS[rc] == code
+
+
+def test_unsupported_head_dim():
+    p = vdn.VdnParams()
+    rc = vdn.lib().vdn_params_init(ctypes.byref(p), 1, 2, 15, 16, 48, 8, vdn.VDN_BF16)
+    assert vdn.STATUS[rc] == "VDN_ERR_UNSUPPORTED"
+
+
+def test_workspace_grows_with_problem():
+    small = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16"))
+    big = vdn.workspace_bytes(vdn.make_params(1, 2, 30, 16, 64, 8, "bf16"))
+    assert 0 < small < big
+    # 768p-shaped workload: transitions, chunk maps, states, V^T, W^T, x
+    p = vdn.make_params(1, 24, 75, 1536, 128, 512, "bf16")
+    ws = vdn.workspace_bytes(p)
+    assert 2.0e9 < ws < 4.0e9
+
+
+def _call_fwd(p, ptrs, ws_ptr, ws_bytes):
+    return vdn.lib().vdn_hybrid_attn_fwd(ctypes.byref(p), *ptrs, ws_ptr, ws_bytes, None)
+
+
+def test_compute_entry_rejects_bad_arguments_before_launch():
+    """Validation errors return before any CUDA call, so they are testable
+    without a device (pointers are never dereferenced on this path)."""
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    need = vdn.workspace_bytes(p)
+    good = [0x10000 + 0x1000 * i for i in range(11)]  # q k v beta alpha tk tv Ws Wl gates out
+    good[4] = None  # alpha may be NULL
+    ws = 0x7f0000000000
+    # missing required pointer
+    bad = list(good)
+    bad[0] = None
+    assert vdn.STATUS[_call_fwd(p, bad, ws, need)] == "VDN_ERR_INVALID_ARG"
+    # misaligned pointer
+    bad = list(good)
+    bad[2] += 8
+    assert vdn.STATUS[_call_fwd(p, bad, ws, need)] == "VDN_ERR_ALIGNMENT"
+    # workspace too small / misaligned / missing
+    assert vdn.STATUS[_call_fwd(p, good, ws, need - 1)] == "VDN_ERR_WORKSPACE"
+    assert vdn.STATUS[_call_fwd(p, good, ws + 16, need)] == "VDN_ERR_ALIGNMENT"
+    assert vdn.STATUS[_call_fwd(p, good, None, need)] == "VDN_ERR_WORKSPACE"
+    # text pointers may be NULL only when n_text == 0
+    bad = list(good)
+    bad[5] = None
+    assert vdn.STATUS[_call_fwd(p, bad, ws, need)] == "VDN_ERR_INVALID_ARG"
+
+
+def test_branches_and_states_validate():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    need = vdn.workspace_bytes(p)
+    L = vdn.lib()
+    rc = L.vdn_hybrid_attn_branches(ctypes.byref(p), None, 0x1000, 0x2000, 0x3000, None, 0x4000,
+                                    0x5000, 0x6000, 0x7000, 0x7f0000000000, need, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"
+    rc = L.vdn_vda_boundary_states(ctypes.byref(p), 0x1000, 0x2000, 0x3000, None, 0x4000, 0x5000,
+                                   0x6008, None, 0x7f0000000000, need, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_ALIGNMENT"
+    assert vdn.STATUS[L.vdn_device_status(ctypes.byref(p), None, None)] == "VDN_ERR_WORKSPACE"

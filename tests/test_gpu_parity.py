@@ -1,0 +1,241 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Small workloads are compared element by element on every output; the
+full-size workloads (768p, long clip, batched clips) are run in the launch
+configuration the benchmark times and compared on seeded samples of query
+rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import softmax_attention_video_chunk_b200 as vdn
+from oracle import vdn_oracle as O
+from synth import CONFIGS, make_inputs, sample_rows
+from tests._parity import TOL_OUT, gpu_rows, oracle_forward, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_ok):
+    return vdn.lib()
+
+
+def _fwd(d, cfg, **kw):
+    return vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                               d["W_soft"], d["W_lin"], d["gates"], cfg.T, alpha=d["alpha"],
+                               chunk=cfg.chunk, window_radius=cfg.window_radius, **kw)
+
+
+def _branches(d, cfg, **kw):
+    return vdn.hybrid_attn_branches(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                                    cfg.T, alpha=d["alpha"], chunk=cfg.chunk,
+                                    window_radius=cfg.window_radius, **kw)
+
+
+# ----------------------------------------------------------------------------
+# full comparison on small workloads
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_tiny_f32_full(simt):
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, simt=simt)
+    o_s, o_l = _branches(d, cfg, simt=simt)
+    F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
+                                   chunk=cfg.chunk)
+    torch.cuda.synchronize()
+    want, ws_, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    assert rel_err(out.double().cpu(), want) <= TOL_OUT["f32"]
+    assert rel_err(o_s.double().cpu(), ws_) <= 1e-5
+    assert rel_err(o_l.double().cpu(), wl_) <= 1e-5
+    Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+                               cfg.T, cfg.N, cfg.chunk)
+    assert rel_err(F.double().cpu(), Fo) <= 1e-5
+    assert rel_err(G.double().cpu(), Go) <= 1e-5
+
+
+@pytest.mark.parametrize("simt", [False, True])
+def test_small_bf16_full(simt):
+    cfg = CONFIGS["small_bf16"]
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, simt=simt)
+    o_s, o_l = _branches(d, cfg, simt=simt)
+    torch.cuda.synchronize()
+    want, ws_, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    e_out = rel_err(out.double().cpu(), want)
+    e_s = rel_err(o_s.double().cpu(), ws_)
+    e_l = rel_err(o_l.double().cpu(), wl_)
+    print(f"small_bf16 simt={simt}: out {e_out:.2e} o_soft {e_s:.2e} o_lin {e_l:.2e}")
+    assert e_out <= TOL_OUT["bf16"]
+    assert e_s <= 2e-3
+    assert e_l <= 1e-4
+
+
+# (name, overrides, make_inputs kwargs, extra fwd kwargs)
+EDGE = [
+    ("T1", dict(T=1, N=40), {}, {}),
+    ("T2", dict(T=2, N=24), {}, {}),
+    ("T7_N5_partial_chunk", dict(T=7, N=5), {}, {}),
+    ("T12_N200_c3_r2", dict(T=12, N=200, chunk=3, window_radius=2), {}, {}),
+    ("T9_N130_c1_r0", dict(T=9, N=130, chunk=1, window_radius=0), {}, {}),
+    ("T23_N96_c4", dict(T=23, N=96, chunk=4), {}, {}),
+    ("no_text", dict(T=16, N=64, n_text=0), {}, {}),
+    ("decay_alpha", dict(T=18, N=48), dict(alpha_range=(0.85, 1.0)), {}),
+    ("text_full", dict(T=16, N=64), {}, dict(text_full=True)),
+    ("d128", dict(T=11, N=136, d=128, H=2), {}, {}),
+    ("d32", dict(T=11, N=40, d=32, H=3), {}, {}),
+]
+
+
+def _edge_cfg(over):
+    base = CONFIGS["small_bf16"].replace(H=3, T=15, N=32, n_text=16, seed=7)
+    return base.replace(**over)
+
+
+def _oracle_inputs_nontext(inp, cfg):
+    if cfg.n_text == 0:
+        B, H, d = cfg.B, cfg.H, cfg.d
+        inp = dict(inp)
+        inp["text_k"] = torch.zeros(B, 0, H, d, dtype=inp["q"].dtype)
+        inp["text_v"] = torch.zeros(B, 0, H, d, dtype=inp["q"].dtype)
+    return inp
+
+
+@pytest.mark.parametrize("simt", [False, True])
+@pytest.mark.parametrize("name,over,mk,kw", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_cases(name, over, mk, kw, simt):
+    cfg = _edge_cfg(over)
+    inp = make_inputs(cfg, **mk)
+    inp = _oracle_inputs_nontext(inp, cfg)
+    d = to_dev(inp)
+    if cfg.n_text == 0:
+        d["text_k"] = d["text_v"] = None
+    out = _fwd(d, cfg, simt=simt, **kw)
+    o_s, o_l = _branches(d, cfg, simt=simt, **kw)
+    torch.cuda.synchronize()
+    want, ws_, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius,
+                                    text_full=kw.get("text_full", False))
+    e_out = rel_err(out.double().cpu(), want)
+    e_s = rel_err(o_s.double().cpu(), ws_)
+    e_l = rel_err(o_l.double().cpu(), wl_)
+    print(f"{name} simt={simt}: out {e_out:.2e} o_soft {e_s:.2e} o_lin {e_l:.2e}")
+    assert e_out <= TOL_OUT["bf16"]
+    assert e_s <= 2e-3
+    assert e_l <= 1e-4
+
+
+def test_wide_scores_rescale_path():
+    """Scores spanning many octaves (q scaled up): the running-max rescale of
+    the tensor-core kernel is exercised."""
+    cfg = _edge_cfg(dict(T=12, N=96, d=64))
+    inp = make_inputs(cfg)
+    inp["q"] = (inp["q"].float() * 40.0).to(torch.bfloat16)
+    d = to_dev(inp)
+    o_s, _ = _branches(d, cfg, want_lin=False)
+    torch.cuda.synchronize()
+    v = O._to_np(inp["v"])
+    ws_ = O.softmax_branch(O._to_np(inp["q"]), O._to_np(inp["k"]), v, cfg.T,
+                           cfg.N, cfg.chunk, cfg.window_radius)
+    # P is rounded once to fp16 (unit roundoff u = 2^-11) before P V, so
+    # |o - o_exact| <= u * sum_j w_j |v_j| <= u * max|v| (weights w sum to 1);
+    # FP32 accumulation adds far less.
+    err = np.max(np.abs(o_s.double().cpu().numpy() - ws_))
+    print(f"wide scores: max|err| {err:.3e}, bound {2.0 ** -11 * np.abs(v).max():.3e}")
+    assert err <= 2.0 ** -11 * np.abs(v).max()
+
+
+def test_out_bf16():
+    cfg = _edge_cfg(dict(T=14, N=64))
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, out_dtype="bf16")
+    torch.cuda.synchronize()
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    # one bf16 rounding of the output on top of the fp32 result
+    want_r = torch.from_numpy(want).to(torch.bfloat16).double().numpy()
+    assert out.dtype == torch.bfloat16
+    err = np.abs(out.double().cpu().numpy() - want_r)
+    ulp = np.abs(want_r) * 2.0 ** -7
+    assert np.all(err <= ulp + 2e-3 * np.sqrt(np.mean(want ** 2)))
+
+
+def test_device_status_ok_and_range():
+    cfg = _edge_cfg(dict(T=10, N=32))
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"])
+    ws = vdn.alloc_workspace(p)
+    _fwd(d, cfg, params=p, workspace=ws)
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"
+    d["v"] = d["v"] * 0 + 1e5  # beyond the fp16 range of the V operand
+    _fwd(d, cfg, params=p, workspace=ws)
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_ERR_RANGE"
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"  # cleared
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads, sampled rows
+# ----------------------------------------------------------------------------
+
+def _sampled(cfg, rows, bsel, chunk=None, **kw):
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    c = cfg.chunk if chunk is None else chunk
+    out = vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                              d["W_soft"], d["W_lin"], d["gates"], cfg.T, chunk=c, **kw)
+    torch.cuda.synchronize()
+    got = gpu_rows(out, rows, bsel)
+    del d, out
+    torch.cuda.empty_cache()
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, c, cfg.window_radius, rows=rows, bsel=bsel)
+    return rel_err(got, want)
+
+
+def test_768p_sampled():
+    cfg = CONFIGS["768p_bf16"]
+    rows = sample_rows(cfg, per_frame=3)
+    e = _sampled(cfg, rows, None)
+    print(f"768p sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_long_clip_sampled():
+    cfg = CONFIGS["long_bf16"]
+    rows = sample_rows(cfg, per_frame=2, chunks=[0, 1, 2, 29, 58, 59])
+    e = _sampled(cfg, rows, None)
+    print(f"long sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_batched_sampled():
+    cfg = CONFIGS["batched_bf16"]
+    rows = sample_rows(cfg, per_frame=3)
+    e = _sampled(cfg, rows, [0, 15])
+    print(f"batched sampled: {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_span_clip_chunk5_and_dense():
+    cfg = CONFIGS["span_bf16"]
+    rows = sample_rows(cfg, per_frame=3)
+    e = _sampled(cfg, rows, [0, 9])
+    assert e <= TOL_OUT["bf16"]
+    # one chunk spanning the clip: the Softmax branch is dense attention
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    o_s, _ = vdn.hybrid_attn_branches(d["q"], d["k"], d["v"], d["beta"], d["text_k"],
+                                      d["text_v"], cfg.T, chunk=cfg.T, want_lin=False)
+    torch.cuda.synchronize()
+    got = gpu_rows(o_s, rows, [3])
+    q = inp["q"][3:4].double()
+    k = inp["k"][3:4].double()
+    v = inp["v"][3:4].double()
+    idx = torch.as_tensor(rows)
+    s = torch.einsum("blhd,bmhd->bhlm", q[:, idx], k) / np.sqrt(cfg.d)
+    dense = torch.einsum("bhlm,bmhd->blhd", torch.softmax(s, dim=-1), v).numpy()
+    assert rel_err(got, dense) <= 2e-3
