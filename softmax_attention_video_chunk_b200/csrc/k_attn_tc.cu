@@ -265,17 +265,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         kv_tile(g, i, k0, lo, hi);
         if (!(ok = wait_bar(s_full + j, i & 1, ab))) break;
         ptx::tc_fence_after();
+        // A tile that lies wholly inside one key range needs no mask.
+        const bool full = (lo == 0 && hi == kBK);
         // pass 1: row maximum over the valid key columns (log2 domain)
         float mx = -INFINITY;
+        if (full) {
+          float mr = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tS + 32 * c, r);
-          ptx::tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tS + 32 * c, r);
+            ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = 32 * c + e;
-            if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(r[e]) * scale_log2);
+            for (int e = 0; e < 32; e += 2)
+              mr = ptx::max3(mr, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+          }
+          mx = mr * scale_log2;  // scale_log2 > 0
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tS + 32 * c, r);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int col = 32 * c + e;
+              if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(r[e]) * scale_log2);
+            }
           }
         }
         if (i == 0) {
@@ -304,30 +320,63 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         // pass 2: P = 2^(s - m) as fp16 pairs over the first 64 columns of S
         float sum = 0.f;
         const float neg_m = -m_used;
+        if (full) {
+          const uint64_t c2 = ptx::f2_pack(scale_log2, scale_log2);
+          const uint64_t nm2 = ptx::f2_pack(neg_m, neg_m);
+          uint64_t acc2 = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t ra[32], rb[32], pk[32];
-          ptx::tmem_ld32(tS + 64 * half, ra);
-          ptx::tmem_ld32(tS + 64 * half + 32, rb);
-          ptx::tmem_wait_ld();
+          for (int half = 0; half < 2; ++half) {
+            uint32_t ra[32], rb[32], pk[32];
+            ptx::tmem_ld32(tS + 64 * half, ra);
+            ptx::tmem_ld32(tS + 64 * half + 32, rb);
+            ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = 64 * half + 2 * e;
-            float p0 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e]), scale_log2, neg_m));
-            float p1 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e + 1]), scale_log2, neg_m));
-            p0 = (c0 >= lo && c0 < hi) ? p0 : 0.f;
-            p1 = (c0 + 1 >= lo && c0 + 1 < hi) ? p1 : 0.f;
-            sum += p0 + p1;
-            pk[e] = pack_half2(p0, p1);
-            const int c1 = c0 + 32;
-            float q0 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e]), scale_log2, neg_m));
-            float q1 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e + 1]), scale_log2, neg_m));
-            q0 = (c1 >= lo && c1 < hi) ? q0 : 0.f;
-            q1 = (c1 + 1 >= lo && c1 + 1 < hi) ? q1 : 0.f;
-            sum += q0 + q1;
-            pk[16 + e] = pack_half2(q0, q1);
+            for (int e = 0; e < 16; ++e) {
+              float x0, x1, y0, y1;
+              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(ra[2 * e]),
+                                                      __uint_as_float(ra[2 * e + 1])), c2, nm2),
+                             x0, x1);
+              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(rb[2 * e]),
+                                                      __uint_as_float(rb[2 * e + 1])), c2, nm2),
+                             y0, y1);
+              const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+              const float q0 = ptx::ex2(y0), q1 = ptx::ex2(y1);
+              acc2 = ptx::f2_add(acc2, ptx::f2_pack(p0, p1));
+              acc2 = ptx::f2_add(acc2, ptx::f2_pack(q0, q1));
+              pk[e] = pack_half2(p0, p1);
+              pk[16 + e] = pack_half2(q0, q1);
+            }
+            ptx::tmem_st32(tS + 32 * half, pk);
           }
-          ptx::tmem_st32(tS + 32 * half, pk);
+          float s0, s1;
+          ptx::f2_unpack(acc2, s0, s1);
+          sum = s0 + s1;
+        } else {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t ra[32], rb[32], pk[32];
+            ptx::tmem_ld32(tS + 64 * half, ra);
+            ptx::tmem_ld32(tS + 64 * half + 32, rb);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = 64 * half + 2 * e;
+              float p0 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e]), scale_log2, neg_m));
+              float p1 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e + 1]), scale_log2, neg_m));
+              p0 = (c0 >= lo && c0 < hi) ? p0 : 0.f;
+              p1 = (c0 + 1 >= lo && c0 + 1 < hi) ? p1 : 0.f;
+              sum += p0 + p1;
+              pk[e] = pack_half2(p0, p1);
+              const int c1 = c0 + 32;
+              float q0 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e]), scale_log2, neg_m));
+              float q1 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e + 1]), scale_log2, neg_m));
+              q0 = (c1 >= lo && c1 < hi) ? q0 : 0.f;
+              q1 = (c1 + 1 >= lo && c1 + 1 < hi) ? q1 : 0.f;
+              sum += q0 + q1;
+              pk[16 + e] = pack_half2(q0, q1);
+            }
+            ptx::tmem_st32(tS + 32 * half, pk);
+          }
         }
         ptx::tmem_wait_st();
         l_sum += sum;

@@ -2,9 +2,6 @@
 //   convert_v   V [B, L, H, D] bf16 -> V^T [B*H][D][Lp] fp16 (keys contiguous:
 //               the K-major B operand of O += P V); zero for keys >= L.
 //   convert_w   [W_soft; W_lin] ([2*H*D][D_out] bf16) -> W^T [D_out][2*H*D] fp16.
-//   readout     linear readout with the decay bridge (FP32), then the RMS
-//               norm and sigmoid gate of the linear branch, written as fp16 into
-//               the right half of the projection operand x.
 //   gemm        out = x W^T on tcgen05 (fp16 operands, FP32 accumulation in
 //               TMEM), TMA-fed 4-stage pipeline, 128 x 256 output tiles.
 // fp16 (11-bit significand) is used for P, V, x and W because bf16 rounding of
@@ -173,138 +170,6 @@ cudaError_t launch_convert_w(const TcFwdArgs& f, cudaStream_t st) {
   convert_w_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)f.W_soft,
                                          (const __nv_bfloat16*)f.W_lin, f.wt, Din, f.D_out,
                                          f.status);
-  return cudaGetLastError();
-}
-
-// --------------------------------------------------------------------------
-// linear readout + bridge + RMS norm + gate -> x[:, H*D + h*D + c] (fp16)
-// --------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256)
-readout_fused_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ alpha,
-                     const float* __restrict__ Rf, const float* __restrict__ FS,
-                     const float* __restrict__ GS, const __nv_bfloat16* __restrict__ gl,
-                     __half* __restrict__ x, int H, int T, int N, int C, int R,
-                     float init_scale, float eps, int* __restrict__ status) {
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int nc = (T + C - 1) / C;
-  const size_t mat = (size_t)D * D;
-  const size_t bh = (size_t)b * H + h;
-  extern __shared__ float smem[];
-  float* Sc = smem;        // [D][D]
-  float* Qs = Sc + D * D;  // [32][D + 1]
-  __shared__ float gf[D], gr[D];
-  const bool anchor = (t == 0 || t == T - 1);
-  const int c = t / C;
-  const int jf = max(0, c - R), jr = min(nc, c + R + 1);
-  const int w0 = max(0, (c - R) * C), w1 = min(T, (c + R + 1) * C);
-  for (int i = tid; i < D; i += blockDim.x) {
-    float a = 1.f, r = 1.f;
-    if (alpha != nullptr && !anchor) {
-      const float* al = alpha + bh * T * D;
-      for (int j = w0; j <= t; ++j) a *= al[(size_t)j * D + i];
-      for (int j = t; j < w1; ++j) r *= al[(size_t)j * D + i];
-    }
-    gf[i] = a;
-    gr[i] = r;
-  }
-  __syncthreads();
-  if (anchor) {
-    const float* St = Rf + (bh * (T + 1)) * mat;
-    for (int e = tid; e < D * D; e += blockDim.x) Sc[e] = 2.f * init_scale * St[e];
-  } else {
-    const float* F = FS + (bh * (nc + 1) + jf) * mat;
-    const float* G = GS + (bh * (nc + 1) + jr) * mat;
-    for (int e = tid; e < D * D; e += blockDim.x) {
-      const int i = e / D;
-      Sc[e] = gf[i] * F[e] + gr[i] * G[e];
-    }
-  }
-  constexpr int NG = D / 32;
-  const int tok = tid >> 3, cg = (tid & 7) * 4;
-  const size_t rs = (size_t)H * D;
-  const size_t L = (size_t)T * N;
-  const size_t row0 = (size_t)b * L + (size_t)t * N;
-  bool bad = false;
-  for (int n0 = 0; n0 < N; n0 += 32) {
-    __syncthreads();
-    for (int e = tid; e < 32 * D; e += blockDim.x) {
-      const int rr = e / D, cc = e % D;
-      Qs[rr * (D + 1) + cc] =
-          (n0 + rr < N) ? __bfloat162float(q[(row0 + n0 + rr) * rs + (size_t)h * D + cc]) : 0.f;
-    }
-    __syncthreads();
-    float acc[NG][4];
-#pragma unroll
-    for (int g = 0; g < NG; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.f;
-    for (int l = 0; l < D; ++l) {
-      const float a = Qs[tok * (D + 1) + l];
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        const float4 sv = *reinterpret_cast<const float4*>(Sc + l * D + cg + 32 * g);
-        acc[g][0] = fmaf(a, sv.x, acc[g][0]);
-        acc[g][1] = fmaf(a, sv.y, acc[g][1]);
-        acc[g][2] = fmaf(a, sv.z, acc[g][2]);
-        acc[g][3] = fmaf(a, sv.w, acc[g][3]);
-      }
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ss = fmaf(acc[g][e], acc[g][e], ss);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-    const float rinv = 1.f / sqrtf(ss / (float)D + eps);
-    if (n0 + tok < N) {
-      const size_t row = row0 + n0 + tok;
-      const __nv_bfloat16* gp = gl + (row * H + h) * D;
-      __half* xp = x + row * (2 * rs) + rs + (size_t)h * D;
-#pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        const int col = cg + 32 * g;
-        const uint2 graw = *reinterpret_cast<const uint2*>(gp + col);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&graw);
-        const float2 ga = __bfloat1622float2(g2[0]), gb = __bfloat1622float2(g2[1]);
-        const float y0 = ga.x * acc[g][0] * rinv, y1 = ga.y * acc[g][1] * rinv;
-        const float y2 = gb.x * acc[g][2] * rinv, y3 = gb.y * acc[g][3] * rinv;
-        bad |= !(fabsf(y0) <= 65504.f) || !(fabsf(y1) <= 65504.f) || !(fabsf(y2) <= 65504.f) ||
-               !(fabsf(y3) <= 65504.f);
-        __half2 h01 = __floats2half2_rn(y0, y1), h23 = __floats2half2_rn(y2, y3);
-        uint2 outv;
-        outv.x = *reinterpret_cast<uint32_t*>(&h01);
-        outv.y = *reinterpret_cast<uint32_t*>(&h23);
-        *reinterpret_cast<uint2*>(xp + col) = outv;
-      }
-    }
-  }
-  if (__syncthreads_or(bad) && tid == 0) atomicOr(status, kDevRange);
-}
-
-cudaError_t launch_readout_tc(const TcFwdArgs& f, cudaStream_t st) {
-  const VdaArgs& a = f.vda;
-  const __nv_bfloat16* gl = (const __nv_bfloat16*)f.gates + (size_t)f.B * f.L * f.H * f.D;
-  cudaError_t e;
-  if (f.D == 128) {
-    const size_t sm = sizeof(float) * (128 * 128 + 32 * 129);
-    if ((e = cudaFuncSetAttribute(readout_fused_kernel<128>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
-      return e;
-    readout_fused_kernel<128><<<dim3(a.T, a.H, a.B), 256, sm, st>>>(
-        (const __nv_bfloat16*)f.q, a.alpha, a.Rf, a.FS, a.GS, gl, f.x, a.H, a.T, a.N, a.C, a.R,
-        a.init_scale, f.eps, f.status);
-  } else if (f.D == 64) {
-    const size_t sm = sizeof(float) * (64 * 64 + 32 * 65);
-    if ((e = cudaFuncSetAttribute(readout_fused_kernel<64>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
-      return e;
-    readout_fused_kernel<64><<<dim3(a.T, a.H, a.B), 256, sm, st>>>(
-        (const __nv_bfloat16*)f.q, a.alpha, a.Rf, a.FS, a.GS, gl, f.x, a.H, a.T, a.N, a.C, a.R,
-        a.init_scale, f.eps, f.status);
-  } else {
-    return cudaErrorInvalidValue;
-  }
   return cudaGetLastError();
 }
 

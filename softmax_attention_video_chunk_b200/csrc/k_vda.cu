@@ -398,7 +398,10 @@ vda_readout_kernel(const TIn* __restrict__ q, const float* __restrict__ alpha,
 template <int D, typename TIn>
 static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
   const int H = a.H, B = a.B, T = a.T, nc = (a.T + a.C - 1) / a.C;
-  {
+  if (a.tc) {
+    cudaError_t e = launch_frame_tc(a, st);
+    if (e != cudaSuccess) return e;
+  } else {
     const size_t sm = sizeof(float) * ((size_t)D * (3 * D + 1) + 2 * 16 * D);
     auto kern = vda_frame_solve_kernel<D, TIn>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

@@ -1,0 +1,325 @@
+// Video Delta Attention frame transitions on the sm_100a tensor cores.
+//
+// "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
+// Generation": per frame, the statistics A_t = beta K_t^T K_t and
+// W_t = beta K_t^T V_t (Video Delta Attention, frame statistics), then the
+// inverse of (I + A_t) in key-channel space and the transition / injection
+// terms M_t = (I + A_t)^-1 Diag(alpha_t), R_t = (I + A_t)^-1 W_t
+// (implementation section, "Small-matrix inverse": Gauss-Jordan elimination
+// held in registers, FP32).
+//
+// One CTA per (b, h, frame); frame 0 is the text virtual frame.
+//   warp 0      TMA producer: 64-token tiles of K and V (bf16, 5-D maps
+//               that stop at the frame edge) into a 3-stage ring;
+//   warp 1      MMA issuer: [K | V]^T-shaped products on tcgen05, both
+//               operands MN-major straight from the TMA tiles:
+//               D[128 x 2d] += K_t^T [K_t | V_t]  (FP32 in TMEM);
+//   all warps   epilogue: D -> shared memory (I + beta A, beta W), then the
+//               in-place Gauss-Jordan inversion of I + beta A with each thread
+//               holding a (d/16) x (d/16) block in registers (one barrier per
+//               pivot), then R = X W and M = X Diag(alpha) on CUDA cores (FP32).
+// For d = 64 the MMA computes [K|V]^T [K|V] (M = N = 128) and keeps the first
+// 64 rows.  Anchor frames write M = Diag(alpha), R = 0 and exit.
+#include "tc_ptx.cuh"
+#include "vdn_common.cuh"
+#include "vdn_kernels.h"
+
+namespace vdn {
+
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v,
+                    const __grid_constant__ CUtensorMap map_tk,
+                    const __grid_constant__ CUtensorMap map_tv, const float* __restrict__ beta,
+                    const float* __restrict__ alpha, float* __restrict__ Mout,
+                    float* __restrict__ Rout, int H, int T, int N, int n_text,
+                    int* __restrict__ status) {
+  constexpr int BT = 64;                  // tokens per stage
+  constexpr int NBLK = D / 32;            // 64-channel blocks of [K | V]
+  constexpr int BLKB = BT * 128;          // bytes of one block (BT rows x 128 B)
+  constexpr int STB = NBLK * BLKB;        // bytes of one stage
+  constexpr int NS = 3;
+  constexpr int NN = 2 * D;               // MMA N (columns of D)
+  constexpr int SD = D + 1;               // padded row stride of the FP32 matrices
+  constexpr int BL = D / 16;              // register block edge per thread
+
+  const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t mat = (size_t)D * D;
+  const size_t bh = (size_t)b * H + h;
+  float* Mo = Mout + (bh * (T + 1) + f) * mat;
+  float* Ro = Rout + (bh * (T + 1) + f) * mat;
+  const int t = f - 1;
+  const float* al = (alpha != nullptr && f >= 1) ? alpha + (bh * T + t) * D : nullptr;
+
+  if (f >= 1 && (t == 0 || t == T - 1)) {  // anchor: decay only, no write
+    for (int e = tid; e < D * D; e += blockDim.x) {
+      const int i = e / D, j = e % D;
+      Mo[e] = (i == j) ? (al ? al[i] : 1.f) : 0.f;
+      Ro[e] = 0.f;
+    }
+    return;
+  }
+  const int ntok = (f == 0) ? n_text : N;
+  const CUtensorMap* mk = (f == 0) ? &map_tk : &map_k;
+  const CUtensorMap* mv = (f == 0) ? &map_tv : &map_v;
+  const int frame_coord = (f == 0) ? 0 : t;
+  const float bt = beta[bh * (T + 1) + f];
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // phase 1: TMA ring; phase 2 (after the MMAs): the two FP32 matrices
+  uint8_t* stages = smem;
+  float* Ash = (float*)smem;           // [D][SD]  I + beta A, then X
+  float* Wsh = Ash + D * SD;           // [D][SD]  beta W
+  constexpr int MATB = 2 * D * SD * 4;
+  constexpr int BIG = (NS * STB > MATB) ? NS * STB : MATB;
+  uint64_t* full = (uint64_t*)(smem + ((BIG + 1023) & ~1023));
+  uint64_t* empty = full + NS;
+  uint64_t* acc_full = empty + NS;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  int* abort_flag = (int*)(tmem_slot + 1);
+  __shared__ float prow[2][D], pcol[2][D];
+
+  const int nst = (ntok + BT - 1) / BT;
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      ptx::mbar_init(full + i, 1);
+      ptx::mbar_init(empty + i, 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 256);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (nst > 0) {
+    if (warp == 0 && lane == 0) {
+      int issued = 0;
+      for (int s = 0; s < nst; ++s) {
+        const int st = s % NS, use = s / NS;
+        if (use > 0 &&
+            !ptx::wait_bounded(empty + st, (use - 1) & 1, abort_flag, status, kDevTimeout))
+          break;
+        ptx::mbar_arrive_expect_tx(full + st, STB);
+        uint8_t* dst = stages + st * STB;
+        for (int kb = 0; kb < D / 64; ++kb)
+          ptx::tma_load_5d(dst + kb * BLKB, mk, full + st, kb * 64, h, s * BT, frame_coord, b);
+        for (int vb = 0; vb < D / 64; ++vb)
+          ptx::tma_load_5d(dst + (D / 64 + vb) * BLKB, mv, full + st, vb * 64, h, s * BT,
+                           frame_coord, b);
+        issued = s + 1;
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = ptx::globaltimer_ns();
+        for (int s = max(0, issued - NS); s < issued; ++s)
+          while (!ptx::mbar_try_wait(full + s % NS, (s / NS) & 1) &&
+                 ptx::globaltimer_ns() - t0 < 2000000000ull) {}
+      }
+    } else if (warp == 1 && lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_f16(128, NN, 1, 1, 1);
+      const uint32_t base = ptx::smem_u32(stages);
+      bool ok = true;
+      for (int s = 0; s < nst; ++s) {
+        const int st = s % NS;
+        if (!(ok = ptx::wait_bounded(full + st, (s / NS) & 1, abort_flag, status, kDevTimeout)))
+          break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk) {
+          const uint32_t a = base + st * STB + kk * 2048;  // 16 token rows of 128 B
+          ptx::mma_ss(tmem, ptx::sdesc_mn_sw128(a, BLKB), ptx::sdesc_mn_sw128(a, BLKB), idesc,
+                      (s > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(empty + st);
+      }
+      if (ok) ptx::mma_commit(acc_full);
+      ptx::mma_commit(drain);
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (!ptx::mbar_try_wait(drain, 0) && ptx::globaltimer_ns() - t0 < 2000000000ull) {}
+    }
+  }
+  // ---- epilogue: D -> shared (all warps) ----
+  bool have = true;
+  if (nst > 0) have = ptx::wait_bounded(acc_full, 0, abort_flag, status, kDevTimeout);
+  __syncthreads();  // every MMA done reading the stages: reuse them for Ash / Wsh
+  ptx::tc_fence_after();
+  {
+    const int q = warp & 3, part = warp >> 2;  // part 0: A columns, 1: W columns
+    const int i = q * 32 + lane;               // row (key channel) = TMEM lane
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + part * D;
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      if (nst > 0 && have) {
+        ptx::tmem_ld32(taddr + 32 * c, r);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (i < D) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = 32 * c + e;
+          const float x = bt * __uint_as_float(r[e]);
+          if (part == 0)
+            Ash[i * SD + j] = x + (i == j ? 1.f : 0.f);
+          else
+            Wsh[i * SD + j] = x;
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 256);
+  }
+
+  // ---- in-place Gauss-Jordan inversion of I + beta A, in registers ----
+  const int ty = tid >> 4, tx = tid & 15;
+  float a[BL][BL];
+#pragma unroll
+  for (int i = 0; i < BL; ++i)
+#pragma unroll
+    for (int c = 0; c < BL; ++c) a[i][c] = Ash[(ty * BL + i) * SD + tx * BL + c];
+  int buf = 0;
+  for (int pb = 0; pb < 16; ++pb) {
+#pragma unroll
+    for (int r = 0; r < BL; ++r) {
+      const int p = pb * BL + r;
+      if (ty == pb) {
+#pragma unroll
+        for (int c = 0; c < BL; ++c) prow[buf][tx * BL + c] = a[r][c];
+      }
+      if (tx == pb) {
+#pragma unroll
+        for (int i = 0; i < BL; ++i) pcol[buf][ty * BL + i] = a[i][r];
+      }
+      __syncthreads();
+      const float piv = 1.f / prow[buf][p];
+      float rp[BL], cp[BL];
+#pragma unroll
+      for (int c = 0; c < BL; ++c) rp[c] = prow[buf][tx * BL + c] * piv;
+#pragma unroll
+      for (int i = 0; i < BL; ++i) cp[i] = pcol[buf][ty * BL + i];
+#pragma unroll
+      for (int i = 0; i < BL; ++i)
+#pragma unroll
+        for (int c = 0; c < BL; ++c) a[i][c] = fmaf(-cp[i], rp[c], a[i][c]);
+      if (ty == pb) {
+#pragma unroll
+        for (int c = 0; c < BL; ++c) a[r][c] = rp[c];
+      }
+      if (tx == pb) {
+#pragma unroll
+        for (int i = 0; i < BL; ++i) a[i][r] = -cp[i] * piv;
+      }
+      if (ty == pb && tx == pb) a[r][r] = piv;
+      buf ^= 1;
+    }
+  }
+  // ---- M = X Diag(alpha) (registers), X -> shared, R = X W ----
+#pragma unroll
+  for (int i = 0; i < BL; ++i) {
+    float* dst = Mo + (size_t)(ty * BL + i) * D + tx * BL;
+#pragma unroll
+    for (int c = 0; c < BL; c += 4) {
+      float4 m4;
+      m4.x = a[i][c] * (al ? al[tx * BL + c] : 1.f);
+      m4.y = a[i][c + 1] * (al ? al[tx * BL + c + 1] : 1.f);
+      m4.z = a[i][c + 2] * (al ? al[tx * BL + c + 2] : 1.f);
+      m4.w = a[i][c + 3] * (al ? al[tx * BL + c + 3] : 1.f);
+      *reinterpret_cast<float4*>(dst + c) = m4;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < BL; ++i)
+#pragma unroll
+    for (int c = 0; c < BL; ++c) Ash[(ty * BL + i) * SD + tx * BL + c] = a[i][c];
+  __syncthreads();
+  float acc[BL][BL];
+#pragma unroll
+  for (int i = 0; i < BL; ++i)
+#pragma unroll
+    for (int c = 0; c < BL; ++c) acc[i][c] = 0.f;
+#pragma unroll 4
+  for (int l = 0; l < D; ++l) {
+    float xv[BL], wv[BL];
+#pragma unroll
+    for (int i = 0; i < BL; ++i) xv[i] = Ash[(ty * BL + i) * SD + l];
+#pragma unroll
+    for (int c = 0; c < BL; ++c) wv[c] = Wsh[l * SD + tx * BL + c];
+#pragma unroll
+    for (int i = 0; i < BL; ++i)
+#pragma unroll
+      for (int c = 0; c < BL; ++c) acc[i][c] = fmaf(xv[i], wv[c], acc[i][c]);
+  }
+#pragma unroll
+  for (int i = 0; i < BL; ++i) {
+    float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
+#pragma unroll
+    for (int c = 0; c < BL; c += 4)
+      *reinterpret_cast<float4*>(dst + c) =
+          make_float4(acc[i][c], acc[i][c + 1], acc[i][c + 2], acc[i][c + 3]);
+  }
+}
+
+template <int D>
+static cudaError_t launch_frame_tc_t(const VdaArgs& a, cudaStream_t st) {
+  CUtensorMap mk, mv, mtk, mtv;
+  const uint64_t Hh = a.H, B = a.B, N = a.N, T = a.T, nt = a.n_text > 0 ? a.n_text : 1;
+  const uint32_t box[5] = {64, 1, 64, 1, 1};
+  {
+    const uint64_t dims[5] = {(uint64_t)D, Hh, N, T, B};
+    const uint64_t str[4] = {(uint64_t)D * 2, Hh * D * 2, N * Hh * D * 2, T * N * Hh * D * 2};
+    if (!make_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.k, dims, str, box) ||
+        !make_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.v, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    // text: one "frame" of n_text tokens; with no text the maps point at k
+    // (never read: the text frame then issues no copy)
+    const void* tk = a.n_text > 0 ? a.text_k : a.k;
+    const void* tv = a.n_text > 0 ? a.text_v : a.v;
+    const uint64_t dims[5] = {(uint64_t)D, Hh, nt, 1, B};
+    const uint64_t str[4] = {(uint64_t)D * 2, Hh * D * 2, nt * Hh * D * 2, nt * Hh * D * 2};
+    if (!make_tmap(&mtk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, tk, dims, str, box) ||
+        !make_tmap(&mtv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, tv, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  constexpr int SD = D + 1;
+  const size_t stage_bytes = 3 * (size_t)(D / 32) * 64 * 128;
+  const size_t mat_bytes = 2 * (size_t)D * SD * 4;
+  const size_t big = ((stage_bytes > mat_bytes ? stage_bytes : mat_bytes) + 1023) & ~(size_t)1023;
+  const size_t sm = 1024 + big + 128;
+  auto kern = vda_frame_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.T + 1, a.H, a.B), 256, sm, st>>>(mk, mv, mtk, mtv, a.beta, a.alpha, a.Mf, a.Rf,
+                                                 a.H, a.T, a.N, a.n_text, a.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_frame_tc(const VdaArgs& a, cudaStream_t st) {
+  if (a.D == 128) return launch_frame_tc_t<128>(a, st);
+  if (a.D == 64) return launch_frame_tc_t<64>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

@@ -118,6 +118,8 @@ static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const
   a.Mf = (float*)(ws + w.Mf); a.Rf = (float*)(ws + w.Rf);
   a.CM = (float*)(ws + w.CM); a.CR = (float*)(ws + w.CR);
   a.FS = (float*)(ws + w.FS); a.GS = (float*)(ws + w.GS);
+  a.tc = use_tc(*p);
+  a.status = (int*)(ws + w.status);
   return a;
 }
 

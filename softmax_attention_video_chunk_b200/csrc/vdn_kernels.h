@@ -16,7 +16,11 @@ struct VdaArgs {
   // workspace: per-frame transitions [B][H][T+1][D][D]; chunk maps
   // [2][B][H][nc][D][D]; boundary states [B][H][nc+1][D][D]
   float *Mf, *Rf, *CM, *CR, *FS, *GS;
+  bool tc;      // frame statistics on the tensor cores (bf16, d in {64, 128})
+  int* status;  // device status word
 };
+
+cudaError_t launch_frame_tc(const VdaArgs& a, cudaStream_t st);
 
 cudaError_t launch_vda_states(const VdaArgs& a, cudaStream_t st);
 cudaError_t launch_vda_readout_simt(const VdaArgs& a, const void* q, float* o_l, cudaStream_t st);

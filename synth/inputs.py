@@ -73,6 +73,10 @@ CONFIGS = {
     # chunk=15 (one chunk, the window spans the clip) for the dense check
     "span_bf16": Config("span_bf16", B=16, H=16, T=15, N=576, d=128,
                         n_text=256, dtype="bf16", seed=4, q_norm=True),
+    # the 768p shape with 4 heads: the profiler workload (inputs > L2, ~1.5 GB
+    # on the device in total)
+    "768p_h4_bf16": Config("768p_h4_bf16", B=1, H=4, T=75, N=1536, d=128, n_text=512,
+                           dtype="bf16", seed=2, q_norm=True),
 }
 
 _TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -239,3 +239,22 @@ def test_span_clip_chunk5_and_dense():
     s = torch.einsum("blhd,bmhd->bhlm", q[:, idx], k) / np.sqrt(cfg.d)
     dense = torch.einsum("bhlm,bmhd->blhd", torch.softmax(s, dim=-1), v).numpy()
     assert rel_err(got, dense) <= 2e-3
+
+
+@pytest.mark.parametrize("over", [dict(T=23, N=96, d=64, H=2), dict(T=12, N=136, d=128, H=2),
+                                  dict(T=9, N=5, d=64, H=2)], ids=["d64", "d128", "N5"])
+def test_boundary_states_tensor_core(over):
+    """Chunk-boundary states of the bf16 path (tensor-core frame statistics +
+    register Gauss-Jordan + chunk composition) against the oracle's literal
+    frame-by-frame recurrence."""
+    cfg = _edge_cfg(over)
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0))
+    d = to_dev(inp)
+    F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
+                                   alpha=d["alpha"], chunk=cfg.chunk)
+    torch.cuda.synchronize()
+    Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+                               cfg.T, cfg.N, cfg.chunk, alpha=inp["alpha"])
+    eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
+    print(f"states {over}: F {eF:.2e} G {eG:.2e}")
+    assert eF <= 1e-4 and eG <= 1e-4
