@@ -54,30 +54,45 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
 }
 
 constexpr int kBK = 128;  // keys per tile
+// Of every 8 (key-pair) exponentials of a full tile, this many are evaluated
+// on the FMA pipe (polynomial) and the rest on the MUFU pipe, so that neither
+// pipe limits the softmax warps.
+#ifndef VDN_KEMU
+#define VDN_KEMU 2
+#endif
+constexpr int kEmu = VDN_KEMU;
 
 // Key tile i of a group: tiles of each key range start at the range start
 // rounded down to 8 tokens (16-byte TMA coordinate of V^T); columns outside
 // [lo, hi) belong to no range of this group and are masked.
 __device__ __forceinline__ void kv_tile(const QGroup& g, int i, int& k0, int& lo, int& hi) {
   k0 = 0; lo = 0; hi = 0;
-  for (int s = 0; s < g.nseg; ++s) {
-    const int a = g.seg0[s] & ~7;
-    const int nt = (g.seg1[s] - a + kBK - 1) / kBK;
-    if (i < nt) {
-      k0 = a + i * kBK;
-      lo = max(g.seg0[s], k0) - k0;
-      hi = min(g.seg1[s], k0 + kBK) - k0;
-      return;
+  bool found = false;
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    if (s < g.nseg && !found) {
+      const int a = g.seg0[s] & ~7;
+      const int nt = (g.seg1[s] - a + kBK - 1) / kBK;
+      if (i < nt) {
+        k0 = a + i * kBK;
+        lo = max(g.seg0[s], k0) - k0;
+        hi = min(g.seg1[s], k0 + kBK) - k0;
+        found = true;
+      } else {
+        i -= nt;
+      }
     }
-    i -= nt;
   }
 }
 
 __device__ __forceinline__ int kv_count(const QGroup& g) {
   int n = 0;
-  for (int s = 0; s < g.nseg; ++s) {
-    const int a = g.seg0[s] & ~7;
-    n += (g.seg1[s] - a + kBK - 1) / kBK;
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    if (s < g.nseg) {
+      const int a = g.seg0[s] & ~7;
+      n += (g.seg1[s] - a + kBK - 1) / kBK;
+    }
   }
   return n;
 }
@@ -265,33 +280,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         kv_tile(g, i, k0, lo, hi);
         if (!(ok = wait_bar(s_full + j, i & 1, ab))) break;
         ptx::tc_fence_after();
-        // A tile that lies wholly inside one key range needs no mask.
-        const bool full = (lo == 0 && hi == kBK);
-        // pass 1: row maximum over the valid key columns (log2 domain)
-        float mx = -INFINITY;
-        if (full) {
-          float mr = -INFINITY;
+        // pass 1: row maximum (all four 32-column loads in flight at once)
+        const bool full = (lo == 0 && hi == kBK);  // tile wholly inside one key range
+        float mx;
+        {
+          uint32_t s[128];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tS + 32 * c, r);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              mr = ptx::max3(mr, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+            uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]);
+            ptx::tmem_ld32(tS + 32 * c, chunk);
           }
-          mx = mr * scale_log2;  // scale_log2 > 0
-        } else {
+          ptx::tmem_wait_ld();
+          if (full) {
+            // eight independent max chains, then a short tree
+            float m8[8];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tS + 32 * c, r);
-            ptx::tmem_wait_ld();
+            for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(s[u]), __uint_as_float(s[8 + u]));
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = 32 * c + e;
-              if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(r[e]) * scale_log2);
-            }
+            for (int e = 16; e < 128; e += 16)
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                m8[u] = ptx::max3(m8[u], __uint_as_float(s[e + u]), __uint_as_float(s[e + 8 + u]));
+            const float mr = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            mx = mr * scale_log2;  // scale_log2 > 0
+          } else {
+            float mr = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              if (e >= lo && e < hi) mr = fmaxf(mr, __uint_as_float(s[e]));
+            mx = mr * scale_log2;
           }
         }
         if (i == 0) {
@@ -317,66 +335,71 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             ptx::tmem_wait_st();
           }
         }
-        // pass 2: P = 2^(s - m) as fp16 pairs over the first 64 columns of S
-        float sum = 0.f;
+        // pass 2: P = 2^(s*scale - m) as fp16 pairs over the first 64 columns of S
         const float neg_m = -m_used;
+        const uint64_t c2 = ptx::f2_pack(scale_log2, scale_log2);
+        const uint64_t nm2 = ptx::f2_pack(neg_m, neg_m);
+        uint64_t acc4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc4[u] = ptx::f2_pack(0.f, 0.f);
         if (full) {
-          const uint64_t c2 = ptx::f2_pack(scale_log2, scale_log2);
-          const uint64_t nm2 = ptx::f2_pack(neg_m, neg_m);
-          uint64_t acc2 = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            uint32_t ra[32], rb[32], pk[32];
+            uint32_t r[64], pk[32];
+            uint32_t (&ra)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+            uint32_t (&rb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
             ptx::tmem_ld32(tS + 64 * half, ra);
             ptx::tmem_ld32(tS + 64 * half + 32, rb);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float x0, x1, y0, y1;
-              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(ra[2 * e]),
-                                                      __uint_as_float(ra[2 * e + 1])), c2, nm2),
-                             x0, x1);
-              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(rb[2 * e]),
-                                                      __uint_as_float(rb[2 * e + 1])), c2, nm2),
-                             y0, y1);
-              const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
-              const float q0 = ptx::ex2(y0), q1 = ptx::ex2(y1);
-              acc2 = ptx::f2_add(acc2, ptx::f2_pack(p0, p1));
-              acc2 = ptx::f2_add(acc2, ptx::f2_pack(q0, q1));
+            for (int e = 0; e < 32; ++e) {
+              const uint64_t x2 = ptx::f2_fma(
+                  ptx::f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), c2, nm2);
+              uint64_t p2;
+              if ((e & 7) < kEmu) {  // FMA-pipe exponentials
+                p2 = ptx::exp2_poly2(x2);
+              } else {               // MUFU exponentials
+                float x0, x1;
+                ptx::f2_unpack(x2, x0, x1);
+                p2 = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
+              }
+              acc4[e & 3] = ptx::f2_add(acc4[e & 3], p2);
+              float p0, p1;
+              ptx::f2_unpack(p2, p0, p1);
               pk[e] = pack_half2(p0, p1);
-              pk[16 + e] = pack_half2(q0, q1);
             }
             ptx::tmem_st32(tS + 32 * half, pk);
           }
-          float s0, s1;
-          ptx::f2_unpack(acc2, s0, s1);
-          sum = s0 + s1;
         } else {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            uint32_t ra[32], rb[32], pk[32];
+            uint32_t r[64], pk[32];
+            uint32_t (&ra)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+            uint32_t (&rb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
             ptx::tmem_ld32(tS + 64 * half, ra);
             ptx::tmem_ld32(tS + 64 * half + 32, rb);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c0 = 64 * half + 2 * e;
-              float p0 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e]), scale_log2, neg_m));
-              float p1 = ptx::ex2(fmaf(__uint_as_float(ra[2 * e + 1]), scale_log2, neg_m));
-              p0 = (c0 >= lo && c0 < hi) ? p0 : 0.f;
-              p1 = (c0 + 1 >= lo && c0 + 1 < hi) ? p1 : 0.f;
-              sum += p0 + p1;
+            for (int e = 0; e < 32; ++e) {
+              const int col = 64 * half + 2 * e;
+              float x0, x1;
+              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(r[2 * e]),
+                                                      __uint_as_float(r[2 * e + 1])), c2, nm2),
+                             x0, x1);
+              const float p0 = (col >= lo && col < hi) ? ptx::ex2(x0) : 0.f;
+              const float p1 = (col + 1 >= lo && col + 1 < hi) ? ptx::ex2(x1) : 0.f;
+              acc4[e & 3] = ptx::f2_add(acc4[e & 3], ptx::f2_pack(p0, p1));
               pk[e] = pack_half2(p0, p1);
-              const int c1 = c0 + 32;
-              float q0 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e]), scale_log2, neg_m));
-              float q1 = ptx::ex2(fmaf(__uint_as_float(rb[2 * e + 1]), scale_log2, neg_m));
-              q0 = (c1 >= lo && c1 < hi) ? q0 : 0.f;
-              q1 = (c1 + 1 >= lo && c1 + 1 < hi) ? q1 : 0.f;
-              sum += q0 + q1;
-              pk[16 + e] = pack_half2(q0, q1);
             }
             ptx::tmem_st32(tS + 32 * half, pk);
           }
+        }
+        float sum;
+        {
+          float s0, s1;
+          ptx::f2_unpack(ptx::f2_add(ptx::f2_add(acc4[0], acc4[1]), ptx::f2_add(acc4[2], acc4[3])),
+                         s0, s1);
+          sum = s0 + s1;
         }
         ptx::tmem_wait_st();
         l_sum += sum;

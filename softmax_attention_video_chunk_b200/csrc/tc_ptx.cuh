@@ -197,6 +197,32 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
+// 2^x for two lanes on the FMA pipe (x <= 64): Cody-Waite style split
+// x = n + f with n = round(x) (exact, via the 1.5 * 2^23 rounding constant) and
+// f in [-1/2, 1/2], 2^f from a degree-4 minimax polynomial (Remez fit of the
+// relative error, max 2.7e-6 with float32 coefficients; fit_exp2_poly.py), and
+// 2^n added into the exponent field.  x is clamped at -125 (2^-125 is zero once
+// rounded to fp16).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t j = f2_add(xc, f2_pack(12582912.f, 12582912.f));
+  const uint64_t n = f2_add(j, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(f2_pack(9.570102207e-03f, 9.570102207e-03f), f,
+                      f2_pack(5.591785908e-02f, 5.591785908e-02f));
+  p = f2_fma(p, f, f2_pack(2.402474433e-01f, 2.402474433e-01f));
+  p = f2_fma(p, f, f2_pack(6.931217909e-01f, 6.931217909e-01f));
+  p = f2_fma(p, f, f2_pack(9.999992847e-01f, 9.999992847e-01f));
+  float p0, p1, j0, j1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(j, j0, j1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23));
+  return f2_pack(r0, r1);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -58,10 +58,16 @@ struct Geo {
     int w0 = (c - R) * C, w1 = (c + R + 1) * C;
     if (w0 < 0) w0 = 0;
     if (w1 > T) w1 = T;
-    q.nseg = 0;
-    if (w0 > 0) { q.seg0[q.nseg] = 0; q.seg1[q.nseg] = N; ++q.nseg; }
-    q.seg0[q.nseg] = w0 * N; q.seg1[q.nseg] = w1 * N; ++q.nseg;
-    if (w1 < T) { q.seg0[q.nseg] = (T - 1) * N; q.seg1[q.nseg] = L; ++q.nseg; }
+    // ranges in increasing order: [anchor 0], window, [anchor T-1]; fixed
+    // slots (no dynamic indexing keeps them in registers)
+    const bool a0 = w0 > 0, a1 = w1 < T;
+    q.seg0[0] = a0 ? 0 : w0 * N;
+    q.seg1[0] = a0 ? N : w1 * N;
+    q.seg0[1] = a0 ? w0 * N : (T - 1) * N;
+    q.seg1[1] = a0 ? w1 * N : L;
+    q.seg0[2] = (T - 1) * N;
+    q.seg1[2] = L;
+    q.nseg = 1 + (a0 ? 1 : 0) + (a1 ? 1 : 0);
     return q;
   }
 };
