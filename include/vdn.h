@@ -184,6 +184,33 @@ VDN_API vdn_status vdn_vda_boundary_states(const vdn_params *p, const void *k, c
                                    float *G, void *workspace, size_t workspace_bytes,
                                    vdn_stream_t stream);
 
+/* Size of the static device array used by vdn_vda_boundary_states_noalloc. */
+#define VDN_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+
+/* vdn_vda_boundary_states without workspace: same kernels, same results, for
+ * callers that cannot allocate device memory (a host framework that owns all
+ * allocations, a plugin with no allocator, code that must not call cudaMalloc
+ * while a stream is captured).  The paper has no counterpart; this is a
+ * deployment convenience of the library.
+ *  - Scratch lives in a static __device__ array of VDN_NOALLOC_SCRATCH_BYTES
+ *    inside the library; each GPU that loads the library keeps it until exit.
+ *    Nothing is allocated or freed by this call.
+ *  - Problems whose state-path scratch exceeds that size return
+ *    VDN_ERR_WORKSPACE.  The scratch is about
+ *    4 * d*d * B*H * (2*(T+1) + 6*ceil(T/chunk) + 2) bytes: e.g. B*H = 8,
+ *    T = 40, d = 64 needs 17 MiB and fits; the 768p workload does not.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents:
+ *    calls that overlap on the GPU (unordered streams or threads) race.  Order
+ *    them on one stream.  The device status word is cleared by each call.
+ *  - Other conventions as vdn_vda_boundary_states; no workspace arguments. */
+VDN_API vdn_status vdn_vda_boundary_states_noalloc(const vdn_params *p, const void *k,
+                                                   const void *v, const float *beta,
+                                                   const float *alpha, const void *text_k,
+                                                   const void *text_v, float *F, float *G,
+                                                   vdn_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device status word that
  * the last compute call on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
  * VDN_ERR_RANGE).  `workspace` must be the one passed to that call. */

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_hybrid_attn_branches.argtypes = [PP] + [_P] * 10 + [ctypes.c_size_t, _P]
         L.vdn_vda_boundary_states.restype = ctypes.c_int
         L.vdn_vda_boundary_states.argtypes = [PP] + [_P] * 9 + [ctypes.c_size_t, _P]
+        L.vdn_vda_boundary_states_noalloc.restype = ctypes.c_int
+        L.vdn_vda_boundary_states_noalloc.argtypes = [PP] + [_P] * 8 + [_P]
         L.vdn_device_status.restype = ctypes.c_int
         L.vdn_device_status.argtypes = [PP, _P, _P]
         _lib = L
@@ -247,6 +249,29 @@ def vda_boundary_states(k, v, beta, text_k, text_v, T, *, alpha=None, workspace=
                                        _ptr(G), _ptr(ws), ws.numel(), _stream(stream))
     if rc != 0:
         raise VdnError(rc, "vdn_vda_boundary_states")
+    return F, G
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def vda_boundary_states_noalloc(k, v, beta, text_k, text_v, T, *, alpha=None, stream=None,
+                                params=None, **kw):
+    """Same result as vda_boundary_states, without any workspace: the library
+    uses its own static device array (NOALLOC_SCRATCH_BYTES per GPU, shared by
+    all calls; calls that overlap on the GPU race).  For callers that cannot
+    allocate device memory.  Only the outputs F, G are allocated here, by the
+    caller side (torch)."""
+    import torch
+    p = params or params_for(k, v, text_k, T, **kw)
+    nc = (p.T + p.chunk - 1) // p.chunk
+    F = torch.empty(p.B, p.H, nc, p.d_k, p.d_v, dtype=torch.float32, device=k.device)
+    G = torch.empty_like(F)
+    rc = lib().vdn_vda_boundary_states_noalloc(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(beta),
+                                               _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(F),
+                                               _ptr(G), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_vda_boundary_states_noalloc")
     return F, G
 
 

@@ -23,6 +23,7 @@ struct WsLayout {
   size_t status, Mf, Rf, CM, CR, FS, GS;   // VDA state path
   size_t o_s, o_l, rinv;                   // CUDA-core path intermediates
   size_t vt, wt, x;                        // tensor-core path operands
+  size_t vda_end;                          // end of the VDA state-path prefix
   size_t total;
 };
 
@@ -46,6 +47,7 @@ static WsLayout layout(const vdn_params& p) {
   w.CR = take(2 * B * H * nc * mat);
   w.FS = take(B * H * (nc + 1) * mat);
   w.GS = take(B * H * (nc + 1) * mat);
+  w.vda_end = off;
   if (use_tc(p)) {
     TcSizes s = tc_sizes(p);
     w.vt = take(s.vt_bytes);
@@ -88,6 +90,15 @@ static vdn_status check_ptr(const void* ptr, bool required) {
   if (ptr == nullptr) return required ? VDN_ERR_INVALID_ARG : VDN_OK;
   return aligned16(ptr) ? VDN_OK : VDN_ERR_ALIGNMENT;
 }
+
+// Bytes of the workspace prefix the VDA state path uses (status word,
+// per-frame transitions, chunk maps, boundary states).
+size_t vda_scratch_bytes(const vdn_params& p) { return layout(p).vda_end; }
+
+vdn_status boundary_states_impl(const vdn_params* p, const void* k, const void* v,
+                                const float* beta, const float* alpha, const void* text_k,
+                                const void* text_v, float* F, float* G, void* workspace,
+                                vdn_stream_t stream);
 
 static vdn_status check_ws(const vdn_params* p, const void* ws, size_t ws_bytes) {
   const WsLayout w = layout(*p);
@@ -203,6 +214,33 @@ vdn_status vdn_vda_boundary_states(const vdn_params* p, const void* k, const voi
   if (F != nullptr || G != nullptr) VDN_CUDA(launch_gather_boundary(a, F, G, st));
   return VDN_OK;
 }
+
+}  // extern "C"
+
+namespace vdn {
+// The boundary-state path of vdn_vda_boundary_states_noalloc: the same
+// launches as vdn_vda_boundary_states on a scratch region whose first
+// vda_scratch_bytes(*p) bytes are usable (checked by the caller).
+vdn_status boundary_states_impl(const vdn_params* p, const void* k, const void* v,
+                                const float* beta, const float* alpha, const void* text_k,
+                                const void* text_v, float* F, float* G, void* workspace,
+                                vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  VDN_TRY(common_inputs(p, nullptr, k, v, beta, alpha, text_k, text_v, false));
+  VDN_TRY(check_ptr(F, false));
+  VDN_TRY(check_ptr(G, false));
+  if (workspace == nullptr) return VDN_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  VdaArgs a = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+  VDN_CUDA(launch_vda_states(a, st));
+  if (F != nullptr || G != nullptr) VDN_CUDA(launch_gather_boundary(a, F, G, st));
+  return VDN_OK;
+}
+}  // namespace vdn
+
+extern "C" {
 
 vdn_status vdn_hybrid_attn_branches(const vdn_params* p, const void* q, const void* k,
                                     const void* v, const float* beta, const float* alpha,
