@@ -161,6 +161,49 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       VDN_TM_IREGS32(r)
       : "memory");
 }
+// Same as tmem_ld32 / tmem_st32 on 32 consecutive elements arr[off .. off+31]
+// of a register array (compile-time indices keep the array in registers).
+#define VDN_R32(a, o)                                                                          \
+  a[o + 0], a[o + 1], a[o + 2], a[o + 3], a[o + 4], a[o + 5], a[o + 6], a[o + 7], a[o + 8],    \
+      a[o + 9], a[o + 10], a[o + 11], a[o + 12], a[o + 13], a[o + 14], a[o + 15], a[o + 16],   \
+      a[o + 17], a[o + 18], a[o + 19], a[o + 20], a[o + 21], a[o + 22], a[o + 23], a[o + 24],  \
+      a[o + 25], a[o + 26], a[o + 27], a[o + 28], a[o + 29], a[o + 30], a[o + 31]
+__device__ __forceinline__ void tmem_ld32_r(
+    uint32_t taddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t& r4,
+    uint32_t& r5, uint32_t& r6, uint32_t& r7, uint32_t& r8, uint32_t& r9, uint32_t& r10,
+    uint32_t& r11, uint32_t& r12, uint32_t& r13, uint32_t& r14, uint32_t& r15, uint32_t& r16,
+    uint32_t& r17, uint32_t& r18, uint32_t& r19, uint32_t& r20, uint32_t& r21, uint32_t& r22,
+    uint32_t& r23, uint32_t& r24, uint32_t& r25, uint32_t& r26, uint32_t& r27, uint32_t& r28,
+    uint32_t& r29, uint32_t& r30, uint32_t& r31) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3), "=r"(r4), "=r"(r5), "=r"(r6), "=r"(r7),
+        "=r"(r8), "=r"(r9), "=r"(r10), "=r"(r11), "=r"(r12), "=r"(r13), "=r"(r14), "=r"(r15),
+        "=r"(r16), "=r"(r17), "=r"(r18), "=r"(r19), "=r"(r20), "=r"(r21), "=r"(r22),
+        "=r"(r23), "=r"(r24), "=r"(r25), "=r"(r26), "=r"(r27), "=r"(r28), "=r"(r29),
+        "=r"(r30), "=r"(r31)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32_r(
+    uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3, uint32_t r4, uint32_t r5,
+    uint32_t r6, uint32_t r7, uint32_t r8, uint32_t r9, uint32_t r10, uint32_t r11, uint32_t r12,
+    uint32_t r13, uint32_t r14, uint32_t r15, uint32_t r16, uint32_t r17, uint32_t r18,
+    uint32_t r19, uint32_t r20, uint32_t r21, uint32_t r22, uint32_t r23, uint32_t r24,
+    uint32_t r25, uint32_t r26, uint32_t r27, uint32_t r28, uint32_t r29, uint32_t r30,
+    uint32_t r31) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7), "r"(r8), "r"(r9),
+      "r"(r10), "r"(r11), "r"(r12), "r"(r13), "r"(r14), "r"(r15), "r"(r16), "r"(r17), "r"(r18),
+      "r"(r19), "r"(r20), "r"(r21), "r"(r22), "r"(r23), "r"(r24), "r"(r25), "r"(r26), "r"(r27),
+      "r"(r28), "r"(r29), "r"(r30), "r"(r31)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
