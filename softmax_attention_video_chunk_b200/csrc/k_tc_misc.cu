@@ -103,25 +103,42 @@ TcFwdArgs tc_fwd_args(const vdn_params& p, const VdaArgs& va, const TcAttnArgs& 
 // --------------------------------------------------------------------------
 // conversions
 // --------------------------------------------------------------------------
+// 64 tokens x D channels per CTA: 16-byte loads along channels into an fp16
+// shared tile, 16-byte stores of 8 consecutive tokens per channel.
 template <int D>
 __global__ void __launch_bounds__(256)
 convert_v_kernel(const __nv_bfloat16* __restrict__ v, __half* __restrict__ vt, int H, int L,
                  int Lp, int* __restrict__ status) {
-  __shared__ float tile[64][D + 1];
+  constexpr int TP = D + 8;  // padded row (halves) of the shared tile
+  __shared__ __align__(16) __half tile[64 * TP];
   const int l0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  for (int e = tid; e < 64 * D; e += blockDim.x) {
-    const int r = e / D, c = e % D, l = l0 + r;
-    tile[r][c] = l < L ? __bfloat162float(v[(((size_t)b * L + l) * H + h) * D + c]) : 0.f;
+  bool bad = false;
+  for (int e = tid; e < 64 * D / 8; e += blockDim.x) {
+    const int r = e / (D / 8), c8 = (e % (D / 8)) * 8, l = l0 + r;
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (l < L) raw = *reinterpret_cast<const uint4*>(v + (((size_t)b * L + l) * H + h) * D + c8);
+    const __nv_bfloat162* in2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    uint4 outv;
+    __half2* out2 = reinterpret_cast<__half2*>(&outv);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(in2[q]);
+      bad |= !(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f);
+      out2[q] = __floats2half2_rn(f.x, f.y);
+    }
+    *reinterpret_cast<uint4*>(&tile[r * TP + c8]) = outv;
   }
   __syncthreads();
-  bool bad = false;
   __half* dst = vt + ((size_t)b * H + h) * D * (size_t)Lp;
-  for (int e = tid; e < 64 * D; e += blockDim.x) {
-    const int c = e >> 6, r = e & 63, l = l0 + r;
+  for (int e = tid; e < D * 8; e += blockDim.x) {
+    // consecutive threads take consecutive channels: conflict-free tile reads
+    const int c = e % D, r8 = (e / D) * 8, l = l0 + r8;
     if (l < Lp) {
-      const float xv = tile[r][c];
-      bad |= !(fabsf(xv) <= 65504.f);
-      dst[(size_t)c * Lp + l] = __float2half_rn(xv);
+      uint4 outv;
+      __half* o = reinterpret_cast<__half*>(&outv);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o[q] = tile[(r8 + q) * TP + c];
+      *reinterpret_cast<uint4*>(dst + (size_t)c * Lp + l) = outv;
     }
   }
   if (__syncthreads_or(bad) && tid == 0) atomicOr(status, kDevRange);
@@ -194,6 +211,10 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile i
 }
 }  // namespace
 
+// Persistent: each CTA walks output tiles t = blockIdx.x, + gridDim.x, ...
+// (n fastest, so consecutive tiles reuse the A row block from L2).  Two TMEM
+// accumulators (2 x 256 columns): the epilogue of one tile overlaps the main
+// loop of the next.
 template <typename TOut>
 __global__ void __launch_bounds__(192, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
@@ -206,25 +227,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   uint8_t* sB = sA + NS * AT;
   uint64_t* full = (uint64_t*)(sB + NS * BT);
   uint64_t* empty = full + NS;
-  uint64_t* acc_full = empty + NS;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* acc_full = empty + NS;   // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2], 128 epilogue arrivals
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   int* abort_flag = (int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int tiles_n = (Nout + BN - 1) / BN;
+  const int ntiles = ((M + BM - 1) / BM) * tiles_n;
   const int nkb = K / BKK;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       ptx::mbar_init(full + i, 1);
       ptx::mbar_init(empty + i, 1);
     }
-    ptx::mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(acc_full + i, 1);
+      ptx::mbar_init(acc_empty + i, 128);
+    }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, 256);
+    ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -236,19 +262,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     if (lane == 0) {
       ptx::prefetch_tmap(&map_x);
       ptx::prefetch_tmap(&map_w);
-      int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int st = kb % NS, use = kb / NS;
-        if (use > 0 && !gwait(empty + st, (use - 1) & 1, abort_flag, status)) break;
-        ptx::mbar_arrive_expect_tx(full + st, AT + BT);
-        ptx::tma_load_2d(sA + st * AT, &map_x, full + st, kb * BKK, m0);
-        ptx::tma_load_2d(sB + st * BT, &map_w, full + st, kb * BKK, n0);
-        issued = kb + 1;
+      int g = 0, issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int st = g % NS, use = g / NS;
+          if (use > 0 &&
+              !(ok = gwait(empty + st, (use - 1) & 1, abort_flag, status)))
+            break;
+          ptx::mbar_arrive_expect_tx(full + st, AT + BT);
+          ptx::tma_load_2d(sA + st * AT, &map_x, full + st, kb * BKK, m0);
+          ptx::tma_load_2d(sB + st * BT, &map_w, full + st, kb * BKK, n0);
+          issued = g + 1;
+        }
       }
       if (*abort_flag) {
         const uint64_t t0 = ptx::globaltimer_ns();
-        for (int kb = max(0, issued - NS); kb < issued; ++kb)
-          while (!ptx::mbar_try_wait(full + kb % NS, (kb / NS) & 1) &&
+        for (int q = max(0, issued - NS); q < issued; ++q)
+          while (!ptx::mbar_try_wait(full + q % NS, (q / NS) & 1) &&
                  ptx::globaltimer_ns() - t0 < kGemmWaitNs) {}
       }
     }
@@ -257,19 +289,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       constexpr uint32_t idesc = ptx::idesc_f16(BM, BN, 0);
       const uint32_t sAa = ptx::smem_u32(sA), sBa = ptx::smem_u32(sB);
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int st = kb % NS;
-        if (!(ok = gwait(full + st, (kb / NS) & 1, abort_flag, status))) break;
+      int g = 0, lt = 0;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        if (lt >= 2 && !(ok = gwait(acc_empty + acc, ((lt >> 1) - 1) & 1, abort_flag, status)))
+          break;
         ptx::tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int st = g % NS;
+          if (!(ok = gwait(full + st, (g / NS) & 1, abort_flag, status))) break;
+          ptx::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BKK / 16; ++kk) {
-          const uint64_t a = ptx::sdesc_k_sw128(sAa + st * AT + kk * 32);
-          const uint64_t bd = ptx::sdesc_k_sw128(sBa + st * BT + kk * 32);
-          ptx::mma_ss(tmem, a, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BKK / 16; ++kk) {
+            const uint64_t a = ptx::sdesc_k_sw128(sAa + st * AT + kk * 32);
+            const uint64_t bd = ptx::sdesc_k_sw128(sBa + st * BT + kk * 32);
+            ptx::mma_ss(d, a, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(empty + st);
         }
-        ptx::mma_commit(empty + st);
+        if (ok) ptx::mma_commit(acc_full + acc);
       }
-      if (ok) ptx::mma_commit(acc_full);
       ptx::mma_commit(drain);
       const uint64_t t0 = ptx::globaltimer_ns();
       while (!ptx::mbar_try_wait(drain, 0) && ptx::globaltimer_ns() - t0 < kGemmWaitNs) {}
@@ -277,10 +317,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   } else {
     // epilogue warps 2..5 -> TMEM lane quarters (warp % 4)
     const int wq = warp & 3;
-    const int m = m0 + wq * 32 + lane;
-    if (gwait(acc_full, 0, abort_flag, status)) {
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!gwait(acc_full + acc, (lt >> 1) & 1, abort_flag, status)) break;
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16);
+      const int m = (t / tiles_n) * BM + wq * 32 + lane, n0 = (t % tiles_n) * BN;
+      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -313,12 +356,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
           }
         }
       }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acc_empty + acc);
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 1) ptx::tmem_dealloc(tmem, 256);
+  if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+static int sm_count() {
+  static int cached[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 cudaError_t launch_gemm_tc(const TcFwdArgs& f, cudaStream_t st) {
@@ -339,7 +397,8 @@ cudaError_t launch_gemm_tc(const TcFwdArgs& f, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   const size_t sm = 1024 + 4 * (128 * 64 * 2) + 4 * (256 * 64 * 2) + 128;
-  const dim3 grid((unsigned)((Nout + 255) / 256), (unsigned)((M + 127) / 128));
+  const uint64_t ntiles = ((Nout + 255) / 256) * ((M + 127) / 128);
+  const dim3 grid((unsigned)(ntiles < (uint64_t)sm_count() ? ntiles : (uint64_t)sm_count()));
   cudaError_t e;
   if (f.out_dtype == VDN_F32) {
     if ((e = cudaFuncSetAttribute(gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
