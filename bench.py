@@ -48,11 +48,13 @@ def visible_frames(t, T, C, R):
     return len(set(range(lo, hi)) | {0, T - 1})
 
 
-def work_model(cfg, out_bytes=4):
+def work_model(cfg, out_bytes=4, text_keys=False):
     B, H, T, N, d, C, R = cfg.B, cfg.H, cfg.T, cfg.N, cfg.d, cfg.chunk, cfg.window_radius
     L, D = T * N, H * d
     frame_pairs = sum(visible_frames(t, T, C, R) for t in range(T))
     pairs = B * H * N * N * frame_pairs              # masked (query, key) pairs
+    if text_keys:
+        pairs += B * H * L * cfg.n_text              # every video query x every text key
     f_soft = 4.0 * d * pairs                          # QK^T and PV
     f_proj = 2.0 * B * L * (2 * D) * D                # [g_s o_s | g_l RMS(o_l)] [W_s; W_l]
     n_fh = B * H * (T + 1)                            # frame-heads incl. the text frame
@@ -63,6 +65,14 @@ def work_model(cfg, out_bytes=4):
                  + 2 * B * cfg.n_text * D * 2 + B * H * (T + 1) * 4)
     return dict(pairs=pairs, frame_pairs=frame_pairs, f_soft=f_soft, f_proj=f_proj,
                 f_vda=f_vda, f_total=f_soft + f_proj + f_vda, bytes_min=bytes_min)
+
+
+# DRAM bytes (read + write) of one attn_tc_kernel launch, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the 4-head copy of the
+# 768p workload: 979.2 MB + 113.0 MB, scaled by the head count (the launch is
+# one independent problem per head).  None for any other workload.
+ATTN_TRAFFIC_PER_HEAD = (979.224064e6 + 112.994816e6) / 4
+ATTN_TRAFFIC_SHAPES = {(75, 1536, 128)}
 
 
 def measured_peaks():
@@ -172,7 +182,9 @@ def base_line(args, cfg, value, ms_per_step, n_gpus):
                    "window_radius": cfg.window_radius, "video_tokens_per_step": cfg.B * cfg.L,
                    "inputs": "seeded synthetic (q,k L2-normalised, v N(0,1), beta sigmoid(N(0,1)), "
                              "gates 0.5, W N(0,1/d)); inputs > L2, no flush",
-                   "out_dtype": "f32", "parallelism": f"replicas x{n_gpus}"},
+                   "out_dtype": "f32", "parallelism": f"replicas x{n_gpus}",
+                   "decay_gate": "U[0.9,1]" if getattr(args, "alpha", False) else "none",
+                   "text_keys_in_softmax": bool(getattr(args, "text_softmax", False))},
     }
 
 
@@ -220,10 +232,10 @@ def run_ours(args, cfg):
         if dist is not None:
             dist.barrier()
 
-    inp = make_inputs(cfg)
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0) if args.alpha else None)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], chunk=cfg.chunk,
-                       window_radius=cfg.window_radius)
+                       window_radius=cfg.window_radius, text_softmax=args.text_softmax)
     ws = vdn.alloc_workspace(p)
     out = torch.empty(cfg.B, cfg.L, p.D_out, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -294,7 +306,7 @@ def run_ours(args, cfg):
     e2e_value = world * tokens * e2e_steps / (e2e_ms / 1e3)
 
     if rank == 0:
-        wm = work_model(cfg)
+        wm = work_model(cfg, text_keys=args.text_softmax)
         pk = measured_peaks()
         soft_ms = stage_ms[2]
         achieved = wm["f_soft"] / (soft_ms / 1e3) / 1e12
@@ -304,7 +316,10 @@ def run_ours(args, cfg):
         line["roofline"] = {
             "bound": "tensor", "kernel": "attn_tc_kernel (window+anchor Softmax)",
             "achieved": achieved, "peak": pk["tc_sust"], "unit": "TFLOP/s",
-            "frac": achieved / pk["tc_sust"], "traffic": None,
+            "frac": achieved / pk["tc_sust"],
+            "traffic": (ATTN_TRAFFIC_PER_HEAD * cfg.B * cfg.H
+                        if (cfg.T, cfg.N, cfg.d) in ATTN_TRAFFIC_SHAPES else None),
+            "traffic_note": "ncu capture of the 4-head 768p shape, scaled by heads",
             "peak_kind": f"{pk['src']} bf16 dense, sustained (kernel timed inside the step loop)",
             "algorithmic_flops_per_launch": wm["f_soft"], "ms_per_launch": soft_ms,
         }
@@ -341,6 +356,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="768p_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--text-softmax", action="store_true",
+                    help="video queries also attend all text tokens in the Softmax branch")
+    ap.add_argument("--alpha", action="store_true",
+                    help="channel-wise decay gate alpha ~ U[0.9, 1] instead of none")
     args = ap.parse_args()
     from synth import CONFIGS
     cfg = CONFIGS[args.config]

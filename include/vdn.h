@@ -97,6 +97,10 @@ typedef struct CUstream_st *vdn_stream_t;
 /* params.flags */
 #define VDN_FLAG_TEXT_FULL (1u << 0) /* both scans start from S_text (not S_text/2) */
 #define VDN_FLAG_SIMT (1u << 1)      /* force the exact-FP32 CUDA-core kernels */
+/* Video queries also attend every text token in the Softmax branch, under one
+ * normaliser with their visible video keys ("text remains directly visible
+ * to the Softmax branch", method section).  Needs n_text > 0. */
+#define VDN_FLAG_TEXT_SOFTMAX (1u << 2)
 
 typedef struct vdn_params {
   int B;             /* batch */

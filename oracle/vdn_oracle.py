@@ -121,12 +121,17 @@ def token_mask(T: int, N: int, chunk: int, radius: int, rows=None) -> np.ndarray
 # ----------------------------------------------------------------------------
 
 def softmax_branch(q, k, v, T, N, chunk=5, radius=1, scale=None, rows=None,
-                   row_block=512):
+                   row_block=512, text_k=None, text_v=None):
     """Exact masked Softmax attention for every (b, h), float64.
 
     o_s[i] = sum_j softmax_j(scale * q_i . k_j  over visible j) v_j, computed
     densely against all L keys with the explicit mask (-inf outside), the row
     maximum subtracted before exp.  ``rows`` selects query tokens.
+
+    With ``text_k`` / ``text_v`` ([B, n_text, H, d]) every video query also
+    sees all text tokens, under the same normaliser ("text remains directly
+    visible to the Softmax branch"; reading: one joint Softmax over the
+    visible video keys and the text keys).
     Returns [B, R, H, d_v].
     """
     q = np.asarray(q, F64)
@@ -135,14 +140,20 @@ def softmax_branch(q, k, v, T, N, chunk=5, radius=1, scale=None, rows=None,
     B, L, H, dk = q.shape
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
+    with_text = text_k is not None and np.asarray(text_k).shape[1] > 0
+    if with_text:
+        k = np.concatenate([k, np.asarray(text_k, F64)], axis=1)
+        v = np.concatenate([v, np.asarray(text_v, F64)], axis=1)
     rows = np.arange(L) if rows is None else np.asarray(rows)
     out = np.zeros((B, len(rows), H, v.shape[-1]), F64)
     for r0 in range(0, len(rows), row_block):
         rr = rows[r0:r0 + row_block]
         mask = token_mask(T, N, chunk, radius, rr)  # [R, L]
+        if with_text:
+            mask = np.concatenate([mask, np.ones((len(rr), k.shape[1] - L), bool)], axis=1)
         for b in range(B):
             for h in range(H):
-                s = scale * (q[b, rr, h, :] @ k[b, :, h, :].T)  # [R, L]
+                s = scale * (q[b, rr, h, :] @ k[b, :, h, :].T)  # [R, L (+ n_text)]
                 s = np.where(mask, s, -np.inf)
                 s = s - s.max(axis=1, keepdims=True)
                 p = np.exp(s)
@@ -310,17 +321,21 @@ def output_projection(o_s, o_l, g_s, g_l, W_soft, W_lin, eps=1e-6):
 
 
 def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
-                   rows=None, text_full=False):
+                   rows=None, text_full=False, text_softmax=False):
     """The whole hybrid attention forward on the selected query rows.
 
     ``inp`` holds numpy (or torch CPU) arrays with the keys q, k, v, beta,
     alpha (or None), text_k, text_v, W_soft, W_lin, gates.
+    ``text_softmax``: video queries also attend all text tokens in the
+    Softmax branch (one normaliser).
     Returns (out [B, R, D_out], o_s [B, R, H, d_v], o_l [B, R, H, d_v]).
     """
     a = {k: (None if v is None else np.asarray(_to_np(v), F64)) for k, v in inp.items()}
     L = a["q"].shape[1]
     rows = np.arange(L) if rows is None else np.asarray(rows)
-    o_s = softmax_branch(a["q"], a["k"], a["v"], T, N, chunk, radius, scale, rows)
+    o_s = softmax_branch(a["q"], a["k"], a["v"], T, N, chunk, radius, scale, rows,
+                         text_k=a["text_k"] if text_softmax else None,
+                         text_v=a["text_v"] if text_softmax else None)
     o_l = linear_branch(a["q"], a["k"], a["v"], a["beta"], a["text_k"], a["text_v"],
                         T, N, chunk, radius, a.get("alpha"), rows, text_full)
     g = a["gates"]

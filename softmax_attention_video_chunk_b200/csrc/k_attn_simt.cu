@@ -21,8 +21,9 @@ namespace vdn {
 template <int D, typename TIn>
 __global__ void __launch_bounds__(128)
 attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
-                 const TIn* __restrict__ v, float* __restrict__ o, Geo geo, int H,
-                 float scale) {
+                 const TIn* __restrict__ v, const TIn* __restrict__ tk,
+                 const TIn* __restrict__ tv, int n_text, float* __restrict__ o, Geo geo,
+                 int H, float scale) {
   constexpr int BQ = 32, BK = 32, QS = D + 4;
   constexpr int NO = D / 16;  // float4 output groups per thread
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -52,15 +53,22 @@ attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 #pragma unroll
   for (int gq = 0; gq < NO; ++gq) acc[gq][0] = acc[gq][1] = acc[gq][2] = acc[gq][3] = 0.f;
 
-  for (int s = 0; s < g.nseg; ++s) {
-    for (int k0 = g.seg0[s]; k0 < g.seg1[s]; k0 += BK) {
-      const int kend = min(BK, g.seg1[s] - k0);
+  // key ranges of the group, then (optionally) the text tokens as one more range
+  const size_t tbase = (size_t)b * n_text * rs + (size_t)h * D;
+  for (int s = 0; s < g.nseg + (n_text > 0 ? 1 : 0); ++s) {
+    const bool text = s == g.nseg;
+    const TIn* ks = text ? tk : k;
+    const TIn* vs = text ? tv : v;
+    const size_t kb = text ? tbase : base;
+    const int s0 = text ? 0 : g.seg0[s], s1 = text ? n_text : g.seg1[s];
+    for (int k0 = s0; k0 < s1; k0 += BK) {
+      const int kend = min(BK, s1 - k0);
       __syncthreads();
       for (int e = tid; e < BK * D; e += blockDim.x) {
         const int rr = e / D, c = e % D;
         const int key = k0 + min(rr, kend - 1);
-        Ks[rr * QS + c] = to_f(k[base + (size_t)key * rs + c]);
-        Vs[rr * D + c] = to_f(v[base + (size_t)key * rs + c]);
+        Ks[rr * QS + c] = to_f(ks[kb + (size_t)key * rs + c]);
+        Vs[rr * D + c] = to_f(vs[kb + (size_t)key * rs + c]);
       }
       __syncthreads();
       // scores for row r, keys sub + 4*m
@@ -136,7 +144,8 @@ static cudaError_t launch_t(const AttnArgs& a, float* o, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   kern<<<dim3(tiles, a.H, a.B), 128, sm, st>>>(
-      (const TIn*)a.q, (const TIn*)a.k, (const TIn*)a.v, o, geo, a.H, a.scale);
+      (const TIn*)a.q, (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.text_k,
+      (const TIn*)a.text_v, a.n_text_keys, o, geo, a.H, a.scale);
   return cudaGetLastError();
 }
 

@@ -97,6 +97,20 @@ __device__ __forceinline__ int kv_count(const QGroup& g) {
   return n;
 }
 
+// Tile i of a query group's key sequence: the group's video key tiles, then
+// (when text keys join the Softmax) ceil(n_text / kBK) tiles of text tokens.
+__device__ __forceinline__ void kv_tile_all(const QGroup& g, int n_video, int n_text, int i,
+                                            int& k0, int& lo, int& hi, bool& text) {
+  text = i >= n_video;
+  if (!text) {
+    kv_tile(g, i, k0, lo, hi);
+  } else {
+    k0 = (i - n_video) * kBK;
+    lo = 0;
+    hi = min(kBK, n_text - k0);
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -107,7 +121,9 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 template <int D, bool FUSED>
 __global__ void __launch_bounds__(320, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-               const __grid_constant__ CUtensorMap map_vt, Geo geo, int B, int H,
+               const __grid_constant__ CUtensorMap map_vt,
+               const __grid_constant__ CUtensorMap map_tk,
+               const __grid_constant__ CUtensorMap map_tvt, int n_text, Geo geo, int B, int H,
                float scale_log2, const __nv_bfloat16* __restrict__ gates,
                __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status) {
   constexpr int BM = 128, NS = 2;
@@ -142,7 +158,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
   if (!find_tile(geo, 2 * BM, pair, &g, &row0)) return;  // uniform over the CTA
   const int row_end = g.row0 + g.nrows;
   const bool has1 = row0 + BM < row_end;
-  const int n_kv = kv_count(g);
+  const int n_video = kv_count(g);
+  const int n_kv = n_video + (n_text + kBK - 1) / kBK;
   const int L = geo.T * geo.N;
 
   if (threadIdx.x == 0) {
@@ -177,6 +194,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
       ptx::prefetch_tmap(&map_q);
       ptx::prefetch_tmap(&map_k);
       ptx::prefetch_tmap(&map_vt);
+      if (n_text > 0) {
+        ptx::prefetch_tmap(&map_tk);
+        ptx::prefetch_tmap(&map_tvt);
+      }
       ptx::mbar_arrive_expect_tx(q_full, (has1 ? 2 : 1) * QT);
       for (int j = 0; j < (has1 ? 2 : 1); ++j)
         for (int sub = 0; sub < NSUB; ++sub)
@@ -187,15 +208,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int st = i % NS, use = i / NS;
         if (use > 0 && !wait_bar(kv_empty + st, (use - 1) & 1, ab)) break;
         int k0, lo, hi;
-        kv_tile(g, i, k0, lo, hi);
+        bool text;
+        kv_tile_all(g, n_video, n_text, i, k0, lo, hi, text);
+        const CUtensorMap* mk = text ? &map_tk : &map_k;
+        const CUtensorMap* mv = text ? &map_tvt : &map_vt;
         ptx::mbar_arrive_expect_tx(k_full + st, KT);
         for (int sub = 0; sub < NSUB; ++sub)
-          ptx::tma_load_4d(sK + st * KT + sub * kBK * 128, &map_k, k_full + st, sub * 64, h, k0,
-                           b);
+          ptx::tma_load_4d(sK + st * KT + sub * kBK * 128, mk, k_full + st, sub * 64, h, k0, b);
         ptx::mbar_arrive_expect_tx(v_full + st, VT);
         for (int vs = 0; vs < 2; ++vs)
-          ptx::tma_load_3d(sV + st * VT + vs * D * 128, &map_vt, v_full + st, k0 + vs * 64, 0,
-                           bh);
+          ptx::tma_load_3d(sV + st * VT + vs * D * 128, mv, v_full + st, k0 + vs * 64, 0, bh);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -277,7 +299,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
       bool ok = true;
       for (int i = 0; i < n_kv; ++i) {
         int k0, lo, hi;
-        kv_tile(g, i, k0, lo, hi);
+        bool text;
+        kv_tile_all(g, n_video, n_text, i, k0, lo, hi, text);
         if (!(ok = wait_bar(s_full + j, i & 1, ab))) break;
         ptx::tc_fence_after();
         // pass 1: row maximum (all four 32-column loads in flight at once)
@@ -483,6 +506,20 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
     if (!make_tmap(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, t.vt, dims, str, box))
       return cudaErrorInvalidValue;
   }
+  CUtensorMap mtk = mk, mtv = mv;  // stand-ins when no text keys (never read)
+  if (t.n_text_keys > 0) {
+    const uint64_t nt = (uint64_t)t.n_text_keys;
+    const uint64_t dims[4] = {(uint64_t)D, H, nt, B};
+    const uint64_t str[3] = {(uint64_t)D * 2, H * D * 2, nt * H * D * 2};
+    const uint32_t box[4] = {64, 1, 128, 1};
+    if (!make_tmap(&mtk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.text_k, dims, str, box))
+      return cudaErrorInvalidValue;
+    const uint64_t dv[3] = {(uint64_t)t.ntp, (uint64_t)D, B * H};
+    const uint64_t sv[2] = {(uint64_t)t.ntp * 2, (uint64_t)D * t.ntp * 2};
+    const uint32_t bv[3] = {64, (uint32_t)D, 1};
+    if (!make_tmap(&mtv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, t.vt_text, dv, sv, bv))
+      return cudaErrorInvalidValue;
+  }
   Geo geo{t.T, t.N, t.C, t.R};
   const int pairs = count_tiles(geo, 256);
   const size_t sm = 1024 + 2 * (128 * D * 2) + 2 * 2 * (128 * D * 2) + 256;
@@ -491,7 +528,7 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
   if (e != cudaSuccess) return e;
   const float scale_log2 = t.scale * 1.4426950408889634f;
   const unsigned grid = (unsigned)pairs * (unsigned)(t.B * t.H);
-  kern<<<grid, 320, sm, st>>>(mq, mk, mv, geo, t.B, t.H, scale_log2,
+  kern<<<grid, 320, sm, st>>>(mq, mk, mv, mtk, mtv, t.n_text_keys, geo, t.B, t.H, scale_log2,
                               FUSED ? (const __nv_bfloat16*)f->gates : nullptr,
                               FUSED ? f->x : nullptr, o_s, t.status);
   return cudaGetLastError();

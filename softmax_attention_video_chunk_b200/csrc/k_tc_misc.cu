@@ -75,7 +75,8 @@ bool use_tc(const vdn_params& p) {
 TcSizes tc_sizes(const vdn_params& p) {
   TcSizes s;
   const size_t L = (size_t)p.T * p.N, Lp = round_up(L, 64);
-  s.vt_bytes = (size_t)p.B * p.H * p.d_k * Lp * 2;
+  const size_t ntp = (p.flags & VDN_FLAG_TEXT_SOFTMAX) ? round_up((size_t)p.n_text, 64) : 0;
+  s.vt_bytes = (size_t)p.B * p.H * p.d_k * (Lp + ntp) * 2;
   s.wt_bytes = (size_t)p.D_out * 2 * p.H * p.d_k * 2;
   s.x_bytes = (size_t)p.B * L * 2 * p.H * p.d_k * 2;
   return s;
@@ -86,6 +87,10 @@ TcAttnArgs tc_attn_args(const vdn_params& p, const AttnArgs& a, void* vt, int* s
   t.B = p.B; t.H = p.H; t.T = p.T; t.N = p.N; t.D = p.d_k; t.C = p.chunk;
   t.R = p.window_radius; t.L = p.T * p.N; t.Lp = (int)round_up((size_t)t.L, 64);
   t.scale = a.scale; t.q = a.q; t.k = a.k; t.v = a.v; t.vt = (__half*)vt; t.status = status;
+  t.n_text_keys = a.n_text_keys;
+  t.ntp = (int)round_up((size_t)a.n_text_keys, 64);
+  t.text_k = a.text_k; t.text_v = a.text_v;
+  t.vt_text = t.vt + (size_t)t.B * t.H * t.D * t.Lp;
   return t;
 }
 
@@ -170,15 +175,22 @@ convert_w_kernel(const __nv_bfloat16* __restrict__ Ws, const __nv_bfloat16* __re
   if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kDevRange);
 }
 
-cudaError_t launch_convert_v(const TcAttnArgs& t, cudaStream_t st) {
-  const dim3 grid(t.Lp / 64, t.H, t.B);
-  if (t.D == 128)
-    convert_v_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)t.v, t.vt, t.H, t.L, t.Lp, t.status);
-  else if (t.D == 64)
-    convert_v_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)t.v, t.vt, t.H, t.L, t.Lp, t.status);
+static cudaError_t convert_one(const void* src, __half* dst, int B, int H, int D, int L, int Lp,
+                               int* status, cudaStream_t st) {
+  const dim3 grid(Lp / 64, H, B);
+  if (D == 128)
+    convert_v_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)src, dst, H, L, Lp, status);
+  else if (D == 64)
+    convert_v_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)src, dst, H, L, Lp, status);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
+}
+
+cudaError_t launch_convert_v(const TcAttnArgs& t, cudaStream_t st) {
+  cudaError_t e = convert_one(t.v, t.vt, t.B, t.H, t.D, t.L, t.Lp, t.status, st);
+  if (e != cudaSuccess || t.n_text_keys == 0) return e;
+  return convert_one(t.text_v, t.vt_text, t.B, t.H, t.D, t.n_text_keys, t.ntp, t.status, st);
 }
 
 cudaError_t launch_convert_w(const TcFwdArgs& f, cudaStream_t st) {

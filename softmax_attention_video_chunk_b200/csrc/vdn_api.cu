@@ -64,7 +64,8 @@ static WsLayout layout(const vdn_params& p) {
 
 static vdn_status validate_params(const vdn_params* p) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;
-  if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT)) return VDN_ERR_INVALID_ARG;
+  if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT | VDN_FLAG_TEXT_SOFTMAX))
+    return VDN_ERR_INVALID_ARG;
   if ((p->dtype != VDN_F32 && p->dtype != VDN_BF16) ||
       (p->out_dtype != VDN_F32 && p->out_dtype != VDN_BF16))
     return VDN_ERR_DTYPE;
@@ -134,12 +135,15 @@ static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const
   return a;
 }
 
-static AttnArgs attn_args(const vdn_params* p, const void* q, const void* k, const void* v) {
+static AttnArgs attn_args(const vdn_params* p, const void* q, const void* k, const void* v,
+                          const void* text_k, const void* text_v) {
   AttnArgs a;
   a.B = p->B; a.H = p->H; a.T = p->T; a.N = p->N; a.D = p->d_k; a.C = p->chunk;
   a.R = p->window_radius; a.dtype = p->dtype;
   a.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.f / sqrtf((float)p->d_k);
   a.q = q; a.k = k; a.v = v;
+  a.n_text_keys = (p->flags & VDN_FLAG_TEXT_SOFTMAX) ? p->n_text : 0;
+  a.text_k = text_k; a.text_v = text_v;
   return a;
 }
 
@@ -263,7 +267,7 @@ vdn_status vdn_hybrid_attn_branches(const vdn_params* p, const void* q, const vo
     VDN_CUDA(launch_vda_readout_simt(a, q, o_lin, st));
   }
   if (o_soft != nullptr) {
-    AttnArgs a = attn_args(p, q, k, v);
+    AttnArgs a = attn_args(p, q, k, v, text_k, text_v);
     if (tc) {
       TcAttnArgs t = tc_attn_args(*p, a, ws + w.vt, (int*)(ws + w.status));
       VDN_CUDA(launch_convert_v(t, st));
@@ -301,7 +305,7 @@ vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const 
   VDN_CUDA(mark(0));
   VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
   VdaArgs va = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
-  AttnArgs aa = attn_args(p, q, k, v);
+  AttnArgs aa = attn_args(p, q, k, v, text_k, text_v);
   if (use_tc(*p)) {
     TcAttnArgs t = tc_attn_args(*p, aa, ws + w.vt, (int*)(ws + w.status));
     TcFwdArgs f = tc_fwd_args(*p, va, t, W_o_soft, W_o_lin, gates, out, ws + w.wt, ws + w.x);

@@ -31,6 +31,8 @@ struct AttnArgs {
   vdn_dtype dtype;
   float scale;
   const void *q, *k, *v;
+  int n_text_keys;                  // text tokens joining the Softmax keys (0: none)
+  const void *text_k, *text_v;      // [B, n_text, H, D]
 };
 cudaError_t launch_attn_simt(const AttnArgs& a, float* o_s, cudaStream_t st);
 

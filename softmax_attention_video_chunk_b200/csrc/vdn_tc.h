@@ -19,6 +19,10 @@ struct TcAttnArgs {
   const void *q, *k, *v;  // bf16 [B, L, H, D]
   __half* vt;             // fp16 [B*H][D][Lp], V transposed (keys contiguous)
   int* status;            // device status word
+  int n_text_keys;        // text tokens joining the Softmax keys (0: none)
+  int ntp;                // n_text_keys rounded up to 64
+  const void *text_k, *text_v;  // bf16 [B, n_text, H, D]
+  __half* vt_text;        // fp16 [B*H][D][ntp], text V transposed
 };
 
 struct TcFwdArgs {

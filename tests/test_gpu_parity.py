@@ -87,6 +87,8 @@ EDGE = [
     ("no_text", dict(T=16, N=64, n_text=0), {}, {}),
     ("decay_alpha", dict(T=18, N=48), dict(alpha_range=(0.85, 1.0)), {}),
     ("text_full", dict(T=16, N=64), {}, dict(text_full=True)),
+    ("text_softmax", dict(T=13, N=72, n_text=200), {}, dict(text_softmax=True)),
+    ("text_softmax_d128", dict(T=9, N=130, d=128, H=2, n_text=77), {}, dict(text_softmax=True)),
     ("d128", dict(T=11, N=136, d=128, H=2), {}, {}),
     ("d32", dict(T=11, N=40, d=32, H=3), {}, {}),
 ]
@@ -119,7 +121,8 @@ def test_edge_cases(name, over, mk, kw, simt):
     o_s, o_l = _branches(d, cfg, simt=simt, **kw)
     torch.cuda.synchronize()
     want, ws_, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius,
-                                    text_full=kw.get("text_full", False))
+                                    text_full=kw.get("text_full", False),
+                                    text_softmax=kw.get("text_softmax", False))
     e_out = rel_err(out.double().cpu(), want)
     e_s = rel_err(o_s.double().cpu(), ws_)
     e_l = rel_err(o_l.double().cpu(), wl_)
@@ -182,12 +185,13 @@ def test_device_status_ok_and_range():
 # full-size workloads, sampled rows
 # ----------------------------------------------------------------------------
 
-def _sampled(cfg, rows, bsel, chunk=None, **kw):
-    inp = make_inputs(cfg)
+def _sampled(cfg, rows, bsel, chunk=None, alpha_range=None, **kw):
+    inp = make_inputs(cfg, alpha_range=alpha_range)
     d = to_dev(inp)
     c = cfg.chunk if chunk is None else chunk
     out = vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                              d["W_soft"], d["W_lin"], d["gates"], cfg.T, chunk=c, **kw)
+                              d["W_soft"], d["W_lin"], d["gates"], cfg.T, chunk=c,
+                              alpha=d["alpha"], **kw)
     torch.cuda.synchronize()
     got = gpu_rows(out, rows, bsel)
     del d, out
@@ -201,6 +205,35 @@ def test_768p_sampled():
     rows = sample_rows(cfg, per_frame=3)
     e = _sampled(cfg, rows, None)
     print(f"768p sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_768p_channel_decay_sampled():
+    """The 768p workload with a channel-wise decay gate alpha ~ U[0.9, 1]
+    (every frame decays the state; the bridge decays across the window)."""
+    cfg = CONFIGS["768p_bf16"]
+    rows = sample_rows(cfg, per_frame=2, chunks=[0, 1, 7, 13, 14])
+    e = _sampled(cfg, rows, None, alpha_range=(0.9, 1.0))
+    print(f"768p decay sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_768p_text_keys_in_softmax_sampled():
+    """The 768p workload with the 512 text tokens joining every video query's
+    Softmax (one normaliser over the visible video keys and the text keys)."""
+    cfg = CONFIGS["768p_bf16"]
+    rows = sample_rows(cfg, per_frame=2, chunks=[0, 7, 14])
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, text_softmax=True)
+    torch.cuda.synchronize()
+    got = gpu_rows(out, rows)
+    del d, out
+    torch.cuda.empty_cache()
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius, rows=rows,
+                                text_softmax=True)
+    e = rel_err(got, want)
+    print(f"768p text-softmax sampled ({len(rows)} rows): {e:.2e}")
     assert e <= TOL_OUT["bf16"]
 
 

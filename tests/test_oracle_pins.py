@@ -362,3 +362,30 @@ def test_projection_head_blocks():
                               np.full((1, 1, 1, 1), 0.5), np.zeros((1, 1, 1, 1)),
                               np.array([[3.0, -1.0]]), np.zeros((1, 2)))
     np.testing.assert_allclose(one, [[[3.0, -1.0]]])
+
+
+def test_softmax_with_text_keys_bruteforce():
+    """Video queries with the text tokens visible: per-row enumeration over
+    the visible video keys plus every text key, one normaliser."""
+    rng = np.random.default_rng(13)
+    B, T, N, H, d, C, nt = 1, 6, 2, 2, 3, 2, 3
+    L = T * N
+    q = rng.normal(size=(B, L, H, d))
+    k = rng.normal(size=(B, L, H, d))
+    v = rng.normal(size=(B, L, H, d))
+    tk = rng.normal(size=(B, nt, H, d))
+    tv = rng.normal(size=(B, nt, H, d))
+    got = O.softmax_branch(q, k, v, T, N, C, 1, text_k=tk, text_v=tv)
+    sc = 1 / np.sqrt(d)
+    for h in range(H):
+        for i in range(L):
+            keys = [(k[0, j, h], v[0, j, h]) for j in range(L)
+                    if _brute_visible(i // N, j // N, T, C, 1)]
+            keys += [(tk[0, t, h], tv[0, t, h]) for t in range(nt)]
+            w = [np.exp(sc * float(np.dot(q[0, i, h], kk))) for kk, _ in keys]
+            want = sum(wi * vv for wi, (_, vv) in zip(w, keys)) / sum(w)
+            np.testing.assert_allclose(got[0, i, h], want, rtol=1e-12, atol=1e-13)
+    # without text keys the result is the plain window+anchor Softmax
+    np.testing.assert_allclose(O.softmax_branch(q, k, v, T, N, C, 1, text_k=tk[:, :0],
+                                                text_v=tv[:, :0]),
+                               O.softmax_branch(q, k, v, T, N, C, 1), rtol=0, atol=0)
