@@ -284,3 +284,76 @@ def device_status(p: VdnParams, workspace, stream=None) -> int:
 def use_tc_params(p: VdnParams) -> bool:
     """True when the call runs the tensor-core kernels (bf16, d in {64, 128})."""
     return p.dtype == VDN_BF16 and p.d_k in (64, 128) and not (p.flags & FLAG_SIMT)
+
+
+class HostPipeline:
+    """End-to-end forwards on host (pinned) tensors with the copies overlapped.
+
+    Each ``submit`` enqueues: host -> device copies of every input (copy
+    stream), the forward (compute stream), and the device -> host copy of
+    ``out`` (copy-back stream), ordered by CUDA events.  Two slots of device
+    buffers alternate, so step i+1's uploads and step i-1's download run while
+    step i computes.  Host input and output tensors must stay untouched until
+    ``synchronize`` (or until the slot is reused two steps later).
+    """
+
+    def __init__(self, host_example: dict, T, *, params=None, **kw):
+        import torch
+        self.T = T
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.dev = dev
+        d0 = {n: (None if host_example.get(n) is None else
+                  torch.empty_like(host_example[n], device=dev)) for n in INPUT_NAMES}
+        self.params = params or params_for(d0["q"], d0["v"], d0["text_k"], T, d0["W_soft"], **kw)
+        p = self.params
+        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
+        self.slots = []
+        for s in range(2):
+            bufs = d0 if s == 0 else {n: (None if v is None else torch.empty_like(v))
+                                      for n, v in d0.items()}
+            out = torch.empty(p.B, p.T * p.N, p.D_out, dtype=odt, device=dev)
+            self.slots.append({"in": bufs, "out": out,
+                               "inputs_free": torch.cuda.Event(), "out_free": torch.cuda.Event(),
+                               "used": False})
+        self.ws = alloc_workspace(p, dev)
+        self.s_h2d = torch.cuda.Stream(dev)
+        self.s_cmp = torch.cuda.Stream(dev)
+        self.s_d2h = torch.cuda.Stream(dev)
+        self.step = 0
+
+    def submit(self, host: dict, out_host):
+        """Enqueue one forward; returns (h2d_bytes, d2h_bytes)."""
+        import torch
+        slot = self.slots[self.step % 2]
+        self.step += 1
+        up, done = torch.cuda.Event(), torch.cuda.Event()
+        h2d = 0
+        with torch.cuda.stream(self.s_h2d):
+            if slot["used"]:
+                self.s_h2d.wait_event(slot["inputs_free"])
+            for n in INPUT_NAMES:
+                if host.get(n) is not None:
+                    slot["in"][n].copy_(host[n], non_blocking=True)
+                    h2d += host[n].numel() * host[n].element_size()
+            up.record(self.s_h2d)
+        with torch.cuda.stream(self.s_cmp):
+            self.s_cmp.wait_event(up)
+            if slot["used"]:
+                self.s_cmp.wait_event(slot["out_free"])
+            d = slot["in"]
+            hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                            d["W_soft"], d["W_lin"], d["gates"], self.T, alpha=d.get("alpha"),
+                            out=slot["out"], workspace=self.ws, stream=self.s_cmp,
+                            params=self.params)
+            slot["inputs_free"].record(self.s_cmp)
+            done.record(self.s_cmp)
+        with torch.cuda.stream(self.s_d2h):
+            self.s_d2h.wait_event(done)
+            out_host.copy_(slot["out"], non_blocking=True)
+            slot["out_free"].record(self.s_d2h)
+        slot["used"] = True
+        return h2d, slot["out"].numel() * slot["out"].element_size()
+
+    def synchronize(self):
+        for s in (self.s_h2d, self.s_cmp, self.s_d2h):
+            s.synchronize()

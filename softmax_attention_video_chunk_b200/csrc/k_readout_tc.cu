@@ -12,7 +12,8 @@
 //   all warps   S_t = Diag(gf_t) F + Diag(gr_t) G (FP32; anchors: S_text), split
 //               into bf16 hi + lo parts (S_hi + S_lo keeps ~16 significant bits
 //               of the FP32 state) and stored as the K-major B operand;
-//   warp 0      TMA producer: 128-token tiles of q (bf16), double-buffered;
+//   warp 0      TMA producer: 128-token tiles of q (bf16), one buffer (two
+//               CTAs share an SM and hide each other's load latency);
 //   warp 1      MMA issuer: O = q S_hi + q S_lo (M = 128 tokens, N = d, FP32
 //               in TMEM, two accumulators);
 //   warps 2-5   epilogue, one token row per thread: RMS over the row, times
@@ -30,7 +31,7 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* b
                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
 readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ alpha,
                   const float* __restrict__ Rf, const float* __restrict__ FS,
                   const float* __restrict__ GS, const __nv_bfloat16* __restrict__ gl,
@@ -50,8 +51,8 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = smem;                 // [hi | lo], each NP panels of [D rows][128 B]
-  uint8_t* sQ = sB + 2 * BTB;         // 2 q tiles
-  uint64_t* q_full = (uint64_t*)(sQ + 2 * QT);
+  uint8_t* sQ = sB + 2 * BTB;         // 1 q tile
+  uint64_t* q_full = (uint64_t*)(sQ + QT);
   uint64_t* q_empty = q_full + 2;
   uint64_t* acc_full = q_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
@@ -118,14 +119,12 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
     if (lane == 0) {
       ptx::prefetch_tmap(&map_q);
       for (int m = 0; m < ntile; ++m) {
-        const int st = m & 1, use = m >> 1;
-        if (use > 0 && !ptx::wait_bounded(q_empty + st, (use - 1) & 1, abort_flag, status,
-                                          kDevTimeout))
+        if (m > 0 &&
+            !ptx::wait_bounded(q_empty, (m - 1) & 1, abort_flag, status, kDevTimeout))
           break;
-        ptx::mbar_arrive_expect_tx(q_full + st, QT);
+        ptx::mbar_arrive_expect_tx(q_full, QT);
         for (int p = 0; p < NP; ++p)
-          ptx::tma_load_4d(sQ + st * QT + p * BM * 128, &map_q, q_full + st, p * 64, h,
-                           t * N + m * BM, b);
+          ptx::tma_load_4d(sQ + p * BM * 128, &map_q, q_full, p * 64, h, t * N + m * BM, b);
       }
     }
   } else if (warp == 1) {
@@ -134,7 +133,7 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
       const uint32_t sQa = ptx::smem_u32(sQ), sBa = ptx::smem_u32(sB);
       for (int m = 0; m < ntile; ++m) {
         const int st = m & 1, use = m >> 1;
-        if (!ptx::wait_bounded(q_full + st, use & 1, abort_flag, status, kDevTimeout)) break;
+        if (!ptx::wait_bounded(q_full, m & 1, abort_flag, status, kDevTimeout)) break;
         if (use > 0 && !ptx::wait_bounded(acc_empty + st, (use - 1) & 1, abort_flag, status,
                                           kDevTimeout))
           break;
@@ -144,13 +143,13 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
         for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * 0 + (kk & 3) * 32;
-            const uint64_t a = ptx::sdesc_k_sw128(sQa + st * QT + (kk >> 2) * (BM * 128) + koff);
+            const uint32_t koff = (kk & 3) * 32;
+            const uint64_t a = ptx::sdesc_k_sw128(sQa + (kk >> 2) * (BM * 128) + koff);
             const uint64_t bd =
                 ptx::sdesc_k_sw128(sBa + part * BTB + (kk >> 2) * (D * 128) + koff);
             ptx::mma_ss(d, a, bd, idesc, (part > 0 || kk > 0) ? 1u : 0u);
           }
-        ptx::mma_commit(q_empty + st);
+        ptx::mma_commit(q_empty);
         ptx::mma_commit(acc_full + st);
       }
       ptx::mma_commit(drain);
@@ -228,7 +227,7 @@ static cudaError_t launch_t(const TcFwdArgs& f, cudaStream_t st) {
   const uint32_t box[4] = {64, 1, 128, 1};
   if (!make_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, f.q, dims, str, box))
     return cudaErrorInvalidValue;
-  const size_t sm = 1024 + 2 * (size_t)D * D * 2 + 2 * 128 * (size_t)D * 2 + 128;
+  const size_t sm = 1024 + 2 * (size_t)D * D * 2 + 128 * (size_t)D * 2 + 128;
   auto kern = readout_tc_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;

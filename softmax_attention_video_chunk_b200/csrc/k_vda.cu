@@ -163,24 +163,29 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
 
 // ---------------------------------------------------------------------------
 // S3: chunk composition.  Forward: frames s..e-1 in increasing order;
-// reverse: e-1..s.  (M, R) <- (M_t M, M_t R + R_t).
+// reverse: e-1..s.  (M, R) <- (M_t M, M_t R + R_t).  Both products act on
+// columns independently, so each CTA composes one 32-column slice of M and R
+// (the whole M_t is staged once per frame).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
 vda_chunk_compose_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf,
                          float* __restrict__ CM, float* __restrict__ CR, int B, int H,
                          int T, int C) {
-  constexpr int RT = D / 16, CT = D / 16, SD = D + 1;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z >> 1, dir = blockIdx.z & 1;
+  constexpr int RT = D / 32, SD = D + 1;
+  const int cb = (blockIdx.x % (D / 32)) * 32;
+  const int c = blockIdx.x / (D / 32);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z >> 1, dir = blockIdx.z & 1;
   const int nc = (T + C - 1) / C;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
   const size_t mat = (size_t)D * D;
   const size_t bh = (size_t)b * H + h;
   const int s = c * C, e = min(T, (c + 1) * C);
   extern __shared__ float smem[];
-  float* Mt = smem;           // [D][SD]
-  float* Ma = Mt + D * SD;    // [D][D]
-  float* Ra = Ma + D * D;     // [D][D]
+  float* Mt = smem;            // [D][SD]
+  float* Ma = Mt + D * SD;     // [D][32]  slice of the composed M
+  float* Ra = Ma + D * 32;     // [D][32]  slice of the composed R
 
   const int nfr = e - s;
   for (int step = 0; step < nfr; ++step) {
@@ -189,54 +194,57 @@ vda_chunk_compose_kernel(const float* __restrict__ Mf, const float* __restrict__
     const float* Rg = Rf + (bh * (T + 1) + 1 + t) * mat;
     __syncthreads();
     if (step == 0) {
-      for (int q = tid; q < D * D; q += blockDim.x) {
-        Ma[q] = Mg[q];
-        Ra[q] = Rg[q];
+      for (int q = tid; q < D * 32; q += blockDim.x) {
+        const int i = q >> 5, j = q & 31;
+        Ma[q] = Mg[i * D + cb + j];
+        Ra[q] = Rg[i * D + cb + j];
       }
       continue;
     }
     for (int q = tid; q < D * D; q += blockDim.x) Mt[(q / D) * SD + (q % D)] = Mg[q];
     __syncthreads();
-    float am[RT][CT], ar[RT][CT];
+    float am[RT][4], ar[RT][4];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
 #pragma unroll
-      for (int m = 0; m < CT; ++m) am[r][m] = ar[r][m] = 0.f;
+      for (int m = 0; m < 4; ++m) am[r][m] = ar[r][m] = 0.f;
 #pragma unroll 4
     for (int l = 0; l < D; ++l) {
-      float a[RT], bm[CT], br[CT];
+      const float4 bm = *reinterpret_cast<const float4*>(Ma + l * 32 + tx * 4);
+      const float4 br = *reinterpret_cast<const float4*>(Ra + l * 32 + tx * 4);
 #pragma unroll
-      for (int r = 0; r < RT; ++r) a[r] = Mt[(ty * RT + r) * SD + l];
-#pragma unroll
-      for (int m = 0; m < CT; ++m) {
-        bm[m] = Ma[l * D + tx + 16 * m];
-        br[m] = Ra[l * D + tx + 16 * m];
+      for (int r = 0; r < RT; ++r) {
+        const float a = Mt[(ty * RT + r) * SD + l];
+        am[r][0] = fmaf(a, bm.x, am[r][0]);
+        am[r][1] = fmaf(a, bm.y, am[r][1]);
+        am[r][2] = fmaf(a, bm.z, am[r][2]);
+        am[r][3] = fmaf(a, bm.w, am[r][3]);
+        ar[r][0] = fmaf(a, br.x, ar[r][0]);
+        ar[r][1] = fmaf(a, br.y, ar[r][1]);
+        ar[r][2] = fmaf(a, br.z, ar[r][2]);
+        ar[r][3] = fmaf(a, br.w, ar[r][3]);
       }
-#pragma unroll
-      for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int m = 0; m < CT; ++m) {
-          am[r][m] = fmaf(a[r], bm[m], am[r][m]);
-          ar[r][m] = fmaf(a[r], br[m], ar[r][m]);
-        }
     }
     __syncthreads();
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
+    for (int r = 0; r < RT; ++r) {
+      const int i = ty * RT + r;
 #pragma unroll
-      for (int m = 0; m < CT; ++m) {
-        const int i = ty * RT + r, j = tx + 16 * m;
-        Ma[i * D + j] = am[r][m];
-        Ra[i * D + j] = ar[r][m] + Rg[i * D + j];
+      for (int m = 0; m < 4; ++m) {
+        const int j = tx * 4 + m;
+        Ma[i * 32 + j] = am[r][m];
+        Ra[i * 32 + j] = ar[r][m] + Rg[i * D + cb + j];
       }
+    }
   }
   __syncthreads();
   // layout [2 (direction)][B][H][nc][D][D]
   float* CMo = CM + ((size_t)dir * B * H * nc + bh * nc + c) * mat;
   float* CRo = CR + ((size_t)dir * B * H * nc + bh * nc + c) * mat;
-  for (int q = tid; q < D * D; q += blockDim.x) {
-    CMo[q] = Ma[q];
-    CRo[q] = Ra[q];
+  for (int q = tid; q < D * 32; q += blockDim.x) {
+    const int i = q >> 5, j = q & 31;
+    CMo[i * D + cb + j] = Ma[q];
+    CRo[i * D + cb + j] = Ra[q];
   }
 }
 
@@ -412,11 +420,11 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
-    const size_t sm = sizeof(float) * ((size_t)D * (D + 1) + 2 * (size_t)D * D);
+    const size_t sm = sizeof(float) * ((size_t)D * (D + 1) + 2 * (size_t)D * 32);
     auto kern = vda_chunk_compose_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(nc, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.CM, a.CR, B, H, T, a.C);
+    kern<<<dim3((D / 32) * nc, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.CM, a.CR, B, H, T, a.C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
