@@ -184,7 +184,9 @@ def base_line(args, cfg, value, ms_per_step, n_gpus):
                              "gates 0.5, W N(0,1/d)); inputs > L2, no flush",
                    "out_dtype": "f32", "parallelism": f"replicas x{n_gpus}",
                    "decay_gate": "U[0.9,1]" if getattr(args, "alpha", False) else "none",
-                   "text_keys_in_softmax": bool(getattr(args, "text_softmax", False))},
+                   "text_keys_in_softmax": bool(getattr(args, "text_softmax", False)),
+                   "write_gate": "per token" if getattr(args, "beta_per_token", False)
+                                 else "per frame"},
     }
 
 
@@ -232,10 +234,12 @@ def run_ours(args, cfg):
         if dist is not None:
             dist.barrier()
 
-    inp = make_inputs(cfg, alpha_range=(0.9, 1.0) if args.alpha else None)
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0) if args.alpha else None,
+                      beta_per_token=args.beta_per_token)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], chunk=cfg.chunk,
-                       window_radius=cfg.window_radius, text_softmax=args.text_softmax)
+                       window_radius=cfg.window_radius, text_softmax=args.text_softmax,
+                       beta_per_token=args.beta_per_token)
     ws = vdn.alloc_workspace(p)
     out = torch.empty(cfg.B, cfg.L, p.D_out, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -366,6 +370,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--text-softmax", action="store_true",
                     help="video queries also attend all text tokens in the Softmax branch")
+    ap.add_argument("--beta-per-token", action="store_true",
+                    help="one write gate per token instead of per frame")
     ap.add_argument("--alpha", action="store_true",
                     help="channel-wise decay gate alpha ~ U[0.9, 1] instead of none")
     args = ap.parse_args()

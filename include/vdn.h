@@ -4,19 +4,19 @@
  *
  * Source of every operation: "Video DeltaNet: A Video-Native Hybrid Attention
  * for Livestream Video Generation" (Xi et al.):
- *   - Softmax branch: the "Nearby frames ..." paragraph of the method (exact
+ *   - Softmax branch: the paragraph of the method on the local window (exact
  *     Softmax inside a chunk-aligned window of 2*window_radius+1 chunks, plus
  *     the two boundary anchors: every frame sees all tokens of the first and
  *     last latent frame, and those two frames see the whole clip; a key frame
  *     counts once).
- *   - Linear branch: the "Bidirectional linear attention ..." paragraph (a
+ *   - Linear branch: the paragraph on bidirectional linear attention (a
  *     forward and a reverse scan over the frames outside the query's window,
  *     anchors excluded, both initialised from a text-summary state, readouts
  *     added; a channel-wise decay bridge across the skipped window span) and
  *     the Video Delta Attention paragraphs (per-frame joint update
  *     S_t = (I + A_t)^-1 (Diag(alpha_t) S_{t-1} + W_t), A_t = beta_t K_t^T K_t,
  *     W_t = beta_t K_t^T V_t, solved in key-channel space, FP32 state).
- *   - Output: the "Both branches receive ..." paragraph (sigmoid gate on the
+ *   - Output: the paragraph on the two output gates (sigmoid gate on the
  *     Softmax readout, RMS norm + sigmoid gate on the linear readout, two
  *     separate output projections whose results are added).
  *   - Implementation section ("Chunk-wise scans", "Small-matrix inverse"):
@@ -30,6 +30,7 @@
  *       q, k, v            [B, L, H, d]      dtype params.dtype
  *       text_k, text_v     [B, n_text, H, d] dtype params.dtype
  *       beta               [B, H, 1+T]       float32; [.,.,0] is the text frame
+ *                          ([B, H, n_text+L] with VDN_FLAG_BETA_PER_TOKEN)
  *       alpha              [B, H, T, d_k]    float32 in [0,1], or NULL (= 1)
  *       W_o_soft, W_o_lin  [H*d_v, D_out]    dtype params.dtype; y = x W
  *       gates              [2, B, L, H, d_v] dtype params.dtype, post-sigmoid;
@@ -98,9 +99,14 @@ typedef struct CUstream_st *vdn_stream_t;
 #define VDN_FLAG_TEXT_FULL (1u << 0) /* both scans start from S_text (not S_text/2) */
 #define VDN_FLAG_SIMT (1u << 1)      /* force the exact-FP32 CUDA-core kernels */
 /* Video queries also attend every text token in the Softmax branch, under one
- * normaliser with their visible video keys ("text remains directly visible
- * to the Softmax branch", method section).  Needs n_text > 0. */
+ * normaliser with their visible video keys (method section: the text keeps
+ * its Softmax path while the linear memory also summarises it).  Needs n_text > 0. */
 #define VDN_FLAG_TEXT_SOFTMAX (1u << 2)
+/* One write gate per token instead of per frame (the pages' beta_{t,i}): beta
+ * is then [B, H, n_text + L] float32, the n_text text tokens first, then the
+ * video tokens in token order.  On the tensor-core path the frame statistics
+ * use sqrt(beta_i)-scaled fp16 copies of the key/value tiles. */
+#define VDN_FLAG_BETA_PER_TOKEN (1u << 3)
 
 typedef struct vdn_params {
   int B;             /* batch */

@@ -8,15 +8,15 @@ Source: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
 Generation" (Xi et al.), method section.  The pages lost every displayed
 equation, so each function states the reading it implements:
 
-* Softmax branch -- "Nearby frames ..." paragraph (chunk-aligned window, the
+* Softmax branch -- the paragraph on the local window (chunk-aligned window, the
   two boundary anchors with four-way connectivity, anchor entries counted
   once).
-* Linear branch -- "Bidirectional linear attention ..." paragraph (forward and
+* Linear branch -- the paragraph on bidirectional linear attention (forward and
   reverse regions outside the window, anchors excluded, decay bridge,
   text-aware initial state counted once) and the Video Delta Attention
   paragraphs (joint objective, normal equation, inverse in key space,
   Proposition 1).
-* Output -- "Both branches receive ..." paragraph (sigmoid gates, RMS norm of
+* Output -- the paragraph on the two output gates (sigmoid gates, RMS norm of
   the linear readout, separate output projections that are added).
 
 Readings where the pages are silent (all are listed with reasons in the
@@ -36,7 +36,8 @@ design notes):
   R11 softmax scale 1/sqrt(d_k); RMS norm over d_v, eps 1e-6, no weight.
 
 Layouts: q, k, v [B, L, H, d] with token index t*N + n; text_k/text_v
-[B, n_text, H, d]; beta [B, H, 1+T] (index 0 = text); alpha [B, H, T, d_k]
+[B, n_text, H, d]; beta [B, H, 1+T] (index 0 = text) per frame, or with
+``beta_per_token`` [B, H, n_text + L] (text tokens first); alpha [B, H, T, d_k]
 or None; gates [2, B, L, H, d_v]; W_soft/W_lin [H*d_v, D_out]; out
 [B, L, D_out].
 """
@@ -53,7 +54,7 @@ F64 = np.float64
 
 def anchor_frames(T: int) -> set:
     """The two boundary anchors: the first and the last latent frame
-    ("Nearby frames ..." paragraph, boundary anchors)."""
+    (the paragraph on the local window, boundary anchors)."""
     return {0, T - 1}
 
 
@@ -69,8 +70,8 @@ def window_frames(t_q: int, T: int, chunk: int, radius: int) -> list:
 def softmax_key_frames(t_q: int, T: int, chunk: int, radius: int) -> list:
     """Key frames visible to query frame t_q in the Softmax branch: an anchor
     query sees every frame; any other query sees its window plus both anchors,
-    each frame once ("Anchor entries already inside a local window are
-    included only once")."""
+    each frame once (method: an anchor frame that also lies in the window
+    is not counted twice)."""
     A = anchor_frames(T)
     if t_q in A:
         return list(range(T))
@@ -129,9 +130,9 @@ def softmax_branch(q, k, v, T, N, chunk=5, radius=1, scale=None, rows=None,
     maximum subtracted before exp.  ``rows`` selects query tokens.
 
     With ``text_k`` / ``text_v`` ([B, n_text, H, d]) every video query also
-    sees all text tokens, under the same normaliser ("text remains directly
-    visible to the Softmax branch"; reading: one joint Softmax over the
-    visible video keys and the text keys).
+    sees all text tokens, under the same normaliser (method: the text keeps
+    its Softmax path; reading: one joint Softmax over the visible video keys
+    and the text keys).
     Returns [B, R, H, d_v].
     """
     q = np.asarray(q, F64)
@@ -167,12 +168,16 @@ def softmax_branch(q, k, v, T, N, chunk=5, radius=1, scale=None, rows=None,
 # ----------------------------------------------------------------------------
 
 def frame_stats(K, V, beta):
-    """Frame statistics of one frame: A = beta K^T K (d_k x d_k) and
-    W = beta K^T V (d_k x d_v); K [n, d_k], V [n, d_v] (Video Delta Attention,
-    frame statistics; write gate per frame, reading R7)."""
+    """Frame statistics of one frame: A = sum_i beta_i k_i k_i^T (d_k x d_k)
+    and W = sum_i beta_i k_i v_i^T (d_k x d_v); K [n, d_k], V [n, d_v]
+    (Video Delta Attention, frame statistics).  ``beta`` is one write gate for
+    the frame (reading R7) or one per token ([n])."""
     K = np.asarray(K, F64)
     V = np.asarray(V, F64)
-    return beta * (K.T @ K), beta * (K.T @ V)
+    if np.ndim(beta) == 0:
+        return beta * (K.T @ K), beta * (K.T @ V)
+    bK = np.asarray(beta, F64)[:, None] * K
+    return K.T @ bK, bK.T @ V
 
 
 def vda_solve(A, W, S_prev, alpha=None):
@@ -204,11 +209,22 @@ def decay(S, alpha):
 
 def text_state(text_k, text_v, beta0):
     """S_text: the text tokens as one leading virtual frame, updated from the
-    zero state ("The linear memory is also text-aware ...")."""
+    zero state (method, the text-aware initial state of both scans)."""
     text_k = np.asarray(text_k, F64)
     text_v = np.asarray(text_v, F64)
     S0 = np.zeros((text_k.shape[1], text_v.shape[1]), F64)
     return vda_update(S0, text_k, text_v, beta0)
+
+
+def _frame_beta(beta_bh, t, N, n_text, per_token):
+    """Write gate(s) of video frame t: beta[1 + t], or its N per-token gates."""
+    if per_token:
+        return beta_bh[n_text + t * N:n_text + (t + 1) * N]
+    return beta_bh[1 + t]
+
+
+def _text_beta(beta_bh, n_text, per_token):
+    return beta_bh[:n_text] if per_token else beta_bh[0]
 
 
 class _FrameStats:
@@ -216,15 +232,17 @@ class _FrameStats:
     the plain definition, so that the literal per-query recurrence below does
     not recompute K_t^T K_t for every query."""
 
-    def __init__(self, k_bh, v_bh, beta_bh, N):
+    def __init__(self, k_bh, v_bh, beta_bh, N, n_text=0, per_token=False):
         self.k, self.v, self.beta, self.N = k_bh, v_bh, beta_bh, N
+        self.n_text, self.per_token = n_text, per_token
         self.cache = {}
 
     def __call__(self, t):
         if t not in self.cache:
             N = self.N
-            self.cache[t] = frame_stats(self.k[t * N:(t + 1) * N],
-                                        self.v[t * N:(t + 1) * N], self.beta[1 + t])
+            self.cache[t] = frame_stats(self.k[t * N:(t + 1) * N], self.v[t * N:(t + 1) * N],
+                                        _frame_beta(self.beta, t, N, self.n_text,
+                                                    self.per_token))
         return self.cache[t]
 
 
@@ -246,9 +264,9 @@ def _scan_outside_window(stats, alpha_bh, init, T, lo, hi):
 
 
 def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
-                  alpha=None, rows=None, text_full=False):
+                  alpha=None, rows=None, text_full=False, beta_per_token=False):
     """Linear (VDA) branch readout o_l = q^T S_f + q^T S_r for every (b, h)
-    ("The distant-context output is the sum of the two readouts").
+    (method: the distant-context output adds the forward and reverse readouts).
 
     For each query chunk the two states are recomputed literally, frame by
     frame, from the text initial state: forward over every frame before the
@@ -271,12 +289,14 @@ def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
     out = np.zeros((B, len(rows), H, dv), F64)
     frames = rows // N
     Aset = anchor_frames(T)
+    nt = text_k.shape[1]
     for b in range(B):
         for h in range(H):
-            S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :], beta[b, h, 0])
+            S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :],
+                                _text_beta(beta[b, h], nt, beta_per_token))
             init = S_text if text_full else 0.5 * S_text
             al = None if alpha is None else np.asarray(alpha, F64)[b, h]
-            stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N)
+            stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N, nt, beta_per_token)
             per_chunk = {}
             for t_q in np.unique(frames):
                 t_q = int(t_q)
@@ -321,7 +341,7 @@ def output_projection(o_s, o_l, g_s, g_l, W_soft, W_lin, eps=1e-6):
 
 
 def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
-                   rows=None, text_full=False, text_softmax=False):
+                   rows=None, text_full=False, text_softmax=False, beta_per_token=False):
     """The whole hybrid attention forward on the selected query rows.
 
     ``inp`` holds numpy (or torch CPU) arrays with the keys q, k, v, beta,
@@ -337,7 +357,7 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
                          text_k=a["text_k"] if text_softmax else None,
                          text_v=a["text_v"] if text_softmax else None)
     o_l = linear_branch(a["q"], a["k"], a["v"], a["beta"], a["text_k"], a["text_v"],
-                        T, N, chunk, radius, a.get("alpha"), rows, text_full)
+                        T, N, chunk, radius, a.get("alpha"), rows, text_full, beta_per_token)
     g = a["gates"]
     out = output_projection(o_s, o_l, g[0][:, rows], g[1][:, rows], a["W_soft"],
                             a["W_lin"], eps)
@@ -345,7 +365,7 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
 
 
 def boundary_states(k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
-                    alpha=None, text_full=False):
+                    alpha=None, text_full=False, beta_per_token=False):
     """For every (b, h) and query chunk c, the forward and reverse states that
     a query of chunk c reads before its bridge: forward = after all frames
     before the window, reverse = after all frames after the window, each
@@ -361,12 +381,14 @@ def boundary_states(k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
     nc = (T + chunk - 1) // chunk
     F = np.zeros((B, H, nc, dk, dv))
     G = np.zeros((B, H, nc, dk, dv))
+    nt = text_k.shape[1]
     for b in range(B):
         for h in range(H):
-            S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :], beta[b, h, 0])
+            S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :],
+                                _text_beta(beta[b, h], nt, beta_per_token))
             init = S_text if text_full else 0.5 * S_text
             al = None if alpha is None else np.asarray(_to_np(alpha), F64)[b, h]
-            stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N)
+            stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N, nt, beta_per_token)
             for c in range(nc):
                 lo = max(0, (c - radius) * chunk)
                 hi = min(T, (c + radius + 1) * chunk)

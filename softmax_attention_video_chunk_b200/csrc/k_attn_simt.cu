@@ -1,7 +1,7 @@
 // Window + anchor Softmax attention on CUDA cores, exact FP32 arithmetic.
 //
 // "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
-// Generation", method, "Nearby frames ..." paragraph: exact Softmax inside the
+// Generation", method, the paragraph on the local window: exact Softmax inside the
 // chunk-aligned window (the query chunk and `radius` chunks on each side), the
 // first and last latent frames visible to every query, and those two frames'
 // queries seeing the whole clip; each key counted once.  The visible keys of a

@@ -1,7 +1,7 @@
 // Window + anchor Softmax attention on the sm_100a tensor cores.
 //
 // "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
-// Generation", method, "Nearby frames ..." paragraph: exact Softmax over the
+// Generation", method, the paragraph on the local window: exact Softmax over the
 // chunk-aligned window plus the two boundary anchors (four-way
 // connectivity), each key once.  The pages run this through a varlen
 // FlashAttention call with queries packed by visible-key pattern; here one

@@ -1,7 +1,7 @@
 // Gated dual output projection on CUDA cores, exact FP32 arithmetic.
 //
 // "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
-// Generation", method, "Both branches receive ..." paragraph: the Softmax
+// Generation", method, the paragraph on the two output gates: the Softmax
 // readout passes its sigmoid gate, the linear readout is RMS-normalised and
 // passes its own sigmoid gate, each branch has its own output projection and
 // the two projections are added:

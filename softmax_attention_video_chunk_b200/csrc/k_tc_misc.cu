@@ -10,7 +10,7 @@
 // reported as VDN_ERR_RANGE through the device status word.
 //
 // Source: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
-// Generation", method ("Both branches receive ..." paragraph: RMS norm and
+// Generation", method (the paragraph on the two output gates: RMS norm and
 // sigmoid gate on the linear readout, separate output projections summed) and
 // implementation ("VDA-Gather", "VDA-Epilogue" fused kernels).
 #include <math.h>

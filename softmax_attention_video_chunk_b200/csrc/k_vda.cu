@@ -36,7 +36,7 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
                        const TIn* __restrict__ text_k, const TIn* __restrict__ text_v,
                        const float* __restrict__ beta, const float* __restrict__ alpha,
                        float* __restrict__ Mout, float* __restrict__ Rout, int H, int T,
-                       int N, int n_text) {
+                       int N, int n_text, bool beta_tok) {
   constexpr int RT = D / 16;  // rows per thread
   constexpr int CT = D / 16;  // cols per thread
   constexpr int BN = 16;      // tokens per staged tile
@@ -72,12 +72,18 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
     V = v + r0 * rs + (size_t)h * D;
     n = N;
   }
-  const float bt = beta[bh * (T + 1) + f];
+  // per-frame gate (scales A and W at the end) or per-token gates (fold into
+  // the staged values)
+  const float bt = beta_tok ? 1.f : beta[bh * (T + 1) + f];
+  const float* btok = beta_tok ? beta + bh * ((size_t)n_text + (size_t)T * N) +
+                                     (f == 0 ? 0 : (size_t)n_text + (size_t)t * N)
+                               : nullptr;
 
   extern __shared__ float smem[];
   float* aug = smem;              // [D][SD]
   float* Ks = aug + D * SD;       // [BN][D]
   float* Vs = Ks + BN * D;        // [BN][D]
+  __shared__ float Bs[BN];
 
   const int ty = tid >> 4, tx = tid & 15;
   float accA[RT][CT], accW[RT][CT];
@@ -94,16 +100,19 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
       Ks[e] = ok ? to_f(K[(size_t)(n0 + rr) * rs + cc]) : 0.f;
       Vs[e] = ok ? to_f(V[(size_t)(n0 + rr) * rs + cc]) : 0.f;
     }
+    for (int rr = tid; rr < BN; rr += blockDim.x)
+      Bs[rr] = (n0 + rr < n) ? (btok ? btok[n0 + rr] : 1.f) : 0.f;
     __syncthreads();
 #pragma unroll 4
     for (int rr = 0; rr < BN; ++rr) {
       float a[RT], kk[CT], vv[CT];
+      const float bn = Bs[rr];
 #pragma unroll
       for (int r = 0; r < RT; ++r) a[r] = Ks[rr * D + ty * RT + r];
 #pragma unroll
       for (int m = 0; m < CT; ++m) {
-        kk[m] = Ks[rr * D + tx + 16 * m];
-        vv[m] = Vs[rr * D + tx + 16 * m];
+        kk[m] = Ks[rr * D + tx + 16 * m] * bn;
+        vv[m] = Vs[rr * D + tx + 16 * m] * bn;
       }
 #pragma unroll
       for (int r = 0; r < RT; ++r)
@@ -416,7 +425,7 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<dim3(T + 1, H, B), 256, sm, st>>>(
         (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.text_k, (const TIn*)a.text_v, a.beta,
-        a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text);
+        a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text, a.beta_tok);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {

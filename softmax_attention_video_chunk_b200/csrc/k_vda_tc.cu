@@ -20,6 +20,11 @@
 //               pivot), then R = X W and M = X Diag(alpha) on CUDA cores (FP32).
 // For d = 64 the MMA computes [K|V]^T [K|V] (M = N = 128) and keeps the first
 // 64 rows.  Anchor frames write M = Diag(alpha), R = 0 and exit.
+// Per-token write gates: warps 2-7 turn every landed bf16 tile into an exact
+// fp16 copy (the A operand, in place) and into beta_i-scaled fp16 hi and lo
+// parts (two B operands: beta*x = hi + lo to ~22 bits); two MMA chains
+// accumulate K^T (beta [K|V])_hi and K^T (beta [K|V])_lo in separate TMEM
+// columns, summed in the epilogue.
 #include "tc_ptx.cuh"
 #include "vdn_common.cuh"
 #include "vdn_kernels.h"
@@ -36,13 +41,16 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_tk,
                     const __grid_constant__ CUtensorMap map_tv, const float* __restrict__ beta,
                     const float* __restrict__ alpha, float* __restrict__ Mout,
-                    float* __restrict__ Rout, int H, int T, int N, int n_text,
+                    float* __restrict__ Rout, int H, int T, int N, int n_text, bool beta_tok,
                     int* __restrict__ status) {
   constexpr int BT = 64;                  // tokens per stage
   constexpr int NBLK = D / 32;            // 64-channel blocks of [K | V]
   constexpr int BLKB = BT * 128;          // bytes of one block (BT rows x 128 B)
-  constexpr int STB = NBLK * BLKB;        // bytes of one stage
-  constexpr int NS = 3;
+  constexpr int STB = NBLK * BLKB;        // bytes of one landed tile
+  // per-frame gates: 3 stages of one tile; per-token gates: 2 stages of three
+  // tiles (A copy, B hi, B lo)
+  const int NS = beta_tok ? 2 : 3;
+  const int SSTR = beta_tok ? 3 * STB : STB;  // stage stride
   constexpr int NN = 2 * D;               // MMA N (columns of D)
   constexpr int SD = D + 1;               // padded row stride of the FP32 matrices
   constexpr int BL = D / 16;              // register block edge per thread
@@ -68,7 +76,10 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   const CUtensorMap* mk = (f == 0) ? &map_tk : &map_k;
   const CUtensorMap* mv = (f == 0) ? &map_tv : &map_v;
   const int frame_coord = (f == 0) ? 0 : t;
-  const float bt = beta[bh * (T + 1) + f];
+  const float bt = beta_tok ? 1.f : beta[bh * (T + 1) + f];
+  const float* btok = beta_tok ? beta + bh * ((size_t)n_text + (size_t)T * N) +
+                                     (f == 0 ? 0 : (size_t)n_text + (size_t)t * N)
+                               : nullptr;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -77,10 +88,12 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   float* Ash = (float*)smem;           // [D][SD]  I + beta A, then X
   float* Wsh = Ash + D * SD;           // [D][SD]  beta W
   constexpr int MATB = 2 * D * SD * 4;
-  constexpr int BIG = (NS * STB > MATB) ? NS * STB : MATB;
+  constexpr int RING = 6 * STB;  // the larger of 3 x STB and 2 x 3 x STB
+  constexpr int BIG = (RING > MATB) ? RING : MATB;
   uint64_t* full = (uint64_t*)(smem + ((BIG + 1023) & ~1023));
-  uint64_t* empty = full + NS;
-  uint64_t* acc_full = empty + NS;
+  uint64_t* empty = full + 3;
+  uint64_t* conv_full = empty + 3;   // per-token gates: operands prepared
+  uint64_t* acc_full = conv_full + 3;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   int* abort_flag = (int*)(tmem_slot + 1);
@@ -88,17 +101,20 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 
   const int nst = (ntok + BT - 1) / BT;
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < 3; ++i) {
       ptx::mbar_init(full + i, 1);
       ptx::mbar_init(empty + i, 1);
+      ptx::mbar_init(conv_full + i, 192);
     }
     ptx::mbar_init(acc_full, 1);
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
+  // per-token gates at d = 128 hold two 256-column accumulators
+  const uint32_t ncols = (beta_tok && 2 * NN > 256) ? 512u : 256u;
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, 256);
+    ptx::tmem_alloc(tmem_slot, ncols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -115,7 +131,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
             !ptx::wait_bounded(empty + st, (use - 1) & 1, abort_flag, status, kDevTimeout))
           break;
         ptx::mbar_arrive_expect_tx(full + st, STB);
-        uint8_t* dst = stages + st * STB;
+        uint8_t* dst = stages + st * SSTR;
         for (int kb = 0; kb < D / 64; ++kb)
           ptx::tma_load_5d(dst + kb * BLKB, mk, full + st, kb * 64, h, s * BT, frame_coord, b);
         for (int vb = 0; vb < D / 64; ++vb)
@@ -130,19 +146,28 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                  ptx::globaltimer_ns() - t0 < 2000000000ull) {}
       }
     } else if (warp == 1 && lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_f16(128, NN, 1, 1, 1);
+      const uint32_t idesc = beta_tok ? ptx::idesc_f16(128, NN, 0, 1, 1)   // fp16 tiles
+                                      : ptx::idesc_f16(128, NN, 1, 1, 1);  // bf16 tiles
       const uint32_t base = ptx::smem_u32(stages);
       bool ok = true;
       for (int s = 0; s < nst; ++s) {
         const int st = s % NS;
-        if (!(ok = ptx::wait_bounded(full + st, (s / NS) & 1, abort_flag, status, kDevTimeout)))
+        if (!(ok = ptx::wait_bounded(beta_tok ? conv_full + st : full + st, (s / NS) & 1,
+                                     abort_flag, status, kDevTimeout)))
           break;
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk) {
-          const uint32_t a = base + st * STB + kk * 2048;  // 16 token rows of 128 B
-          ptx::mma_ss(tmem, ptx::sdesc_mn_sw128(a, BLKB), ptx::sdesc_mn_sw128(a, BLKB), idesc,
-                      (s > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t a = base + st * SSTR + kk * 2048;  // 16 token rows of 128 B
+          const uint64_t ad = ptx::sdesc_mn_sw128(a, BLKB);
+          if (!beta_tok) {
+            ptx::mma_ss(tmem, ad, ad, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            ptx::mma_ss(tmem, ad, ptx::sdesc_mn_sw128(a + STB, BLKB), idesc,
+                        (s > 0 || kk > 0) ? 1u : 0u);
+            ptx::mma_ss(tmem + NN, ad, ptx::sdesc_mn_sw128(a + 2 * STB, BLKB), idesc,
+                        (s > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         ptx::mma_commit(empty + st);
       }
@@ -150,6 +175,44 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
       ptx::mma_commit(drain);
       const uint64_t t0 = ptx::globaltimer_ns();
       while (!ptx::mbar_try_wait(drain, 0) && ptx::globaltimer_ns() - t0 < 2000000000ull) {}
+    } else if (beta_tok && warp >= 2) {
+      // rescale each landed tile: row r of a 64-token block is token s*BT + r
+      const int ct = tid - 64;  // 0..191
+      bool bad = false;
+      for (int s = 0; s < nst; ++s) {
+        const int st = s % NS;
+        if (!ptx::wait_bounded(full + st, (s / NS) & 1, abort_flag, status, kDevTimeout)) break;
+        uint8_t* base = stages + st * SSTR;
+        for (int ch = ct; ch < STB / 16; ch += 192) {
+          const int off = ch * 16;
+          const int row = (off % BLKB) / 128;
+          const int tok = s * BT + row;
+          const float bw = tok < ntok ? btok[tok] : 0.f;
+          const uint4 raw = *reinterpret_cast<const uint4*>(base + off);
+          const __nv_bfloat162* in2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          uint4 av, hv, lv;
+          __half2* a2 = reinterpret_cast<__half2*>(&av);
+          __half2* h2 = reinterpret_cast<__half2*>(&hv);
+          __half2* l2 = reinterpret_cast<__half2*>(&lv);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 x = __bfloat1622float2(in2[q]);
+            const float y0 = x.x * bw, y1 = x.y * bw;
+            bad |= !(fabsf(x.x) <= 65504.f) || !(fabsf(x.y) <= 65504.f) ||
+                   !(fabsf(y0) <= 65504.f) || !(fabsf(y1) <= 65504.f);
+            a2[q] = __floats2half2_rn(x.x, x.y);  // exact for bf16 in the fp16 range
+            h2[q] = __floats2half2_rn(y0, y1);
+            const float2 hf = __half22float2(h2[q]);
+            l2[q] = __floats2half2_rn(y0 - hf.x, y1 - hf.y);
+          }
+          *reinterpret_cast<uint4*>(base + off) = av;
+          *reinterpret_cast<uint4*>(base + STB + off) = hv;
+          *reinterpret_cast<uint4*>(base + 2 * STB + off) = lv;
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(conv_full + st);
+      }
+      if (bad) atomicOr(status, kDevRange);
     }
   }
   // ---- epilogue: D -> shared (all warps) ----
@@ -166,6 +229,14 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
       if (nst > 0 && have) {
         ptx::tmem_ld32(taddr + 32 * c, r);
         ptx::tmem_wait_ld();
+        if (beta_tok) {  // add the lo-part accumulator
+          uint32_t r2[32];
+          ptx::tmem_ld32(taddr + NN + 32 * c, r2);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(r2[e]));
+        }
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0u;
@@ -187,7 +258,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 256);
+    ptx::tmem_dealloc(tmem, ncols);
   }
 
   // ---- in-place Gauss-Jordan inversion of I + beta A, in registers ----
@@ -304,7 +375,7 @@ static cudaError_t launch_frame_tc_t(const VdaArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   constexpr int SD = D + 1;
-  const size_t stage_bytes = 3 * (size_t)(D / 32) * 64 * 128;
+  const size_t stage_bytes = 6 * (size_t)(D / 32) * 64 * 128;
   const size_t mat_bytes = 2 * (size_t)D * SD * 4;
   const size_t big = ((stage_bytes > mat_bytes ? stage_bytes : mat_bytes) + 1023) & ~(size_t)1023;
   const size_t sm = 1024 + big + 128;
@@ -312,7 +383,7 @@ static cudaError_t launch_frame_tc_t(const VdaArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.T + 1, a.H, a.B), 256, sm, st>>>(mk, mv, mtk, mtv, a.beta, a.alpha, a.Mf, a.Rf,
-                                                 a.H, a.T, a.N, a.n_text, a.status);
+                                                 a.H, a.T, a.N, a.n_text, a.beta_tok, a.status);
   return cudaGetLastError();
 }
 

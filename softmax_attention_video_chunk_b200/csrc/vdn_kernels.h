@@ -17,6 +17,7 @@ struct VdaArgs {
   // [2][B][H][nc][D][D]; boundary states [B][H][nc+1][D][D]
   float *Mf, *Rf, *CM, *CR, *FS, *GS;
   bool tc;      // frame statistics on the tensor cores (bf16, d in {64, 128})
+  bool beta_tok;  // beta per token: [B][H][n_text + L]
   int* status;  // device status word
 };
 

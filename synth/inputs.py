@@ -18,7 +18,9 @@ distributions with a seeded CPU generator, in a fixed order:
 All draws are float32; the result is then rounded once to the workload dtype
 (round-to-nearest-even for bf16).  alpha (the decay gate) is None for the
 standard workloads (alpha == 1); ``alpha_range`` draws alpha ~ U[lo, hi]
-per (b, h, frame, channel) as an extra, final draw.
+per (b, h, frame, channel) as an extra draw after the gates;
+``beta_per_token`` then draws one write gate per token,
+sigmoid(N(0, 1)) [B, H, n_text + L] (text tokens first), replacing beta.
 
 L = T * N and token index = t * N + n (frame-major, token-minor).
 """
@@ -87,7 +89,7 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_inputs(cfg: Config, *, alpha_range: Optional[tuple] = None,
-                beta_override: Optional[torch.Tensor] = None,
+                beta_override: Optional[torch.Tensor] = None, beta_per_token: bool = False,
                 device: str = "cpu") -> dict:
     """Draw one workload.  Returns torch tensors in the workload dtype
     (beta, alpha always float32) on ``device``.
@@ -124,6 +126,8 @@ def make_inputs(cfg: Config, *, alpha_range: Optional[tuple] = None,
         out["alpha"] = lo + (hi - lo) * u
     else:
         out["alpha"] = None
+    if beta_per_token:
+        out["beta"] = torch.sigmoid(randn(B, H, cfg.n_text + L))
     if device != "cpu":
         out = {k: (v.to(device) if v is not None else None) for k, v in out.items()}
     return out

@@ -89,6 +89,10 @@ EDGE = [
     ("text_full", dict(T=16, N=64), {}, dict(text_full=True)),
     ("text_softmax", dict(T=13, N=72, n_text=200), {}, dict(text_softmax=True)),
     ("text_softmax_d128", dict(T=9, N=130, d=128, H=2, n_text=77), {}, dict(text_softmax=True)),
+    ("beta_per_token", dict(T=14, N=72), dict(beta_per_token=True, alpha_range=(0.9, 1.0)),
+     dict(beta_per_token=True)),
+    ("beta_per_token_d128_N5", dict(T=8, N=5, d=128, H=2, n_text=37),
+     dict(beta_per_token=True), dict(beta_per_token=True)),
     ("d128", dict(T=11, N=136, d=128, H=2), {}, {}),
     ("d32", dict(T=11, N=40, d=32, H=3), {}, {}),
 ]
@@ -122,7 +126,8 @@ def test_edge_cases(name, over, mk, kw, simt):
     torch.cuda.synchronize()
     want, ws_, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius,
                                     text_full=kw.get("text_full", False),
-                                    text_softmax=kw.get("text_softmax", False))
+                                    text_softmax=kw.get("text_softmax", False),
+                                    beta_per_token=kw.get("beta_per_token", False))
     e_out = rel_err(out.double().cpu(), want)
     e_s = rel_err(o_s.double().cpu(), ws_)
     e_l = rel_err(o_l.double().cpu(), wl_)
@@ -237,6 +242,24 @@ def test_768p_text_keys_in_softmax_sampled():
     assert e <= TOL_OUT["bf16"]
 
 
+def test_768p_per_token_beta_sampled():
+    """The 768p workload with one write gate per token, sigmoid(N(0,1))."""
+    cfg = CONFIGS["768p_bf16"]
+    rows = sample_rows(cfg, per_frame=2, chunks=[0, 7, 14])
+    inp = make_inputs(cfg, beta_per_token=True)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, beta_per_token=True)
+    torch.cuda.synchronize()
+    got = gpu_rows(out, rows)
+    del d, out
+    torch.cuda.empty_cache()
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius, rows=rows,
+                                beta_per_token=True)
+    e = rel_err(got, want)
+    print(f"768p per-token beta sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
 def test_long_clip_sampled():
     cfg = CONFIGS["long_bf16"]
     rows = sample_rows(cfg, per_frame=2, chunks=[0, 1, 2, 29, 58, 59])
@@ -274,20 +297,22 @@ def test_span_clip_chunk5_and_dense():
     assert rel_err(got, dense) <= 2e-3
 
 
+@pytest.mark.parametrize("beta_tok", [False, True])
 @pytest.mark.parametrize("over", [dict(T=23, N=96, d=64, H=2), dict(T=12, N=136, d=128, H=2),
                                   dict(T=9, N=5, d=64, H=2)], ids=["d64", "d128", "N5"])
-def test_boundary_states_tensor_core(over):
+def test_boundary_states_tensor_core(over, beta_tok):
     """Chunk-boundary states of the bf16 path (tensor-core frame statistics +
     register Gauss-Jordan + chunk composition) against the oracle's literal
     frame-by-frame recurrence."""
     cfg = _edge_cfg(over)
-    inp = make_inputs(cfg, alpha_range=(0.9, 1.0))
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0), beta_per_token=beta_tok)
     d = to_dev(inp)
     F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
-                                   alpha=d["alpha"], chunk=cfg.chunk)
+                                   alpha=d["alpha"], chunk=cfg.chunk, beta_per_token=beta_tok)
     torch.cuda.synchronize()
     Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
-                               cfg.T, cfg.N, cfg.chunk, alpha=inp["alpha"])
+                               cfg.T, cfg.N, cfg.chunk, alpha=inp["alpha"],
+                               beta_per_token=beta_tok)
     eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
     print(f"states {over}: F {eF:.2e} G {eG:.2e}")
     assert eF <= 1e-4 and eG <= 1e-4

@@ -172,7 +172,7 @@ def test_token_mask_expands_frames():
 
 def test_window_is_15_frames_inside_clip():
     """A query chunk away from the ends attends 3 chunks = 15 frames
-    ("producing a 15-frame window except at sequence boundaries")."""
+    (method, local window: 15 frames wherever the clip does not cut it)."""
     T = 75
     assert len(O.window_frames(37, T, 5, 1)) == 15
     assert len(O.window_frames(2, T, 5, 1)) == 10       # shrunk at the start
@@ -389,3 +389,31 @@ def test_softmax_with_text_keys_bruteforce():
     np.testing.assert_allclose(O.softmax_branch(q, k, v, T, N, C, 1, text_k=tk[:, :0],
                                                 text_v=tv[:, :0]),
                                O.softmax_branch(q, k, v, T, N, C, 1), rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_per_token_beta_least_squares(seed):
+    """Per-token write gates: the update minimises
+    1/2||S - S~||^2 + 1/2 sum_i beta_i ||S^T k_i - v_i||^2 (stacked rows sqrt(beta_i))."""
+    rng = np.random.default_rng(400 + seed)
+    dk, dv, n = 6, 5, 9
+    S_prev = rng.normal(size=(dk, dv))
+    K = _unit(rng.normal(size=(n, dk)))
+    V = rng.normal(size=(n, dv))
+    beta = rng.uniform(0.0, 2.0, size=n)
+    alpha = rng.uniform(0.5, 1.0, size=dk)
+    Amat = np.vstack([np.eye(dk), np.sqrt(beta)[:, None] * K])
+    rhs = np.vstack([alpha[:, None] * S_prev, np.sqrt(beta)[:, None] * V])
+    want = np.linalg.lstsq(Amat, rhs, rcond=None)[0]
+    np.testing.assert_allclose(O.vda_update(S_prev, K, V, beta, alpha), want,
+                               rtol=1e-10, atol=1e-10)
+
+
+def test_per_token_beta_constant_equals_per_frame():
+    q, k, v, tk, tv, beta, alpha = _tiny_linear_inputs(26)
+    T, N, nt = 17, 3, 5
+    per_tok = np.concatenate([np.repeat(beta[:, :, :1], nt, axis=2),
+                              np.repeat(beta[:, :, 1:], N, axis=2)], axis=2)
+    a = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1, alpha=alpha)
+    b = O.linear_branch(q, k, v, per_tok, tk, tv, T, N, 5, 1, alpha=alpha, beta_per_token=True)
+    np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
