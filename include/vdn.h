@@ -226,6 +226,21 @@ VDN_API vdn_status vdn_vda_boundary_states_noalloc(const vdn_params *p, const vo
  * VDN_ERR_RANGE).  `workspace` must be the one passed to that call. */
 VDN_API vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_stream_t stream);
 
+/* Self-test of failure detection, without a fault or a hang.
+ * Every pipelined kernel of this library bounds its waits on shared-memory
+ * barriers by time: on expiry it records VDN_ERR_TIMEOUT in the device status
+ * word, the other warps of the block leave through an abort flag, and the
+ * block frees its tensor memory and exits.  This call enqueues one block that
+ * runs that sequence on a barrier nothing ever arrives at.
+ *  - workspace: any workspace of this library (device memory, 256-byte
+ *    aligned); only its status word is written.  It is cleared first, so
+ *    vdn_device_status afterwards returns VDN_ERR_TIMEOUT.
+ *  - limit_us: the wait limit, 100 us .. 1 s (else VDN_ERR_INVALID_ARG).  The
+ *    block ends within about twice this limit.
+ *  - The GPU context stays usable; later calls run normally. */
+VDN_API vdn_status vdn_selftest_bounded_wait(void *workspace, unsigned int limit_us,
+                                             vdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_vda_boundary_states_noalloc.argtypes = [PP] + [_P] * 8 + [_P]
         L.vdn_device_status.restype = ctypes.c_int
         L.vdn_device_status.argtypes = [PP, _P, _P]
+        L.vdn_selftest_bounded_wait.restype = ctypes.c_int
+        L.vdn_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint, _P]
         _lib = L
     return _lib
 
@@ -281,6 +283,11 @@ def vda_boundary_states_noalloc(k, v, beta, text_k, text_v, T, *, alpha=None, st
 def device_status(p: VdnParams, workspace, stream=None) -> int:
     """Synchronise and return (and clear) the device status of the last call."""
     return lib().vdn_device_status(ctypes.byref(p), _ptr(workspace), _stream(stream))
+
+
+def selftest_bounded_wait(workspace, limit_us: int, stream=None) -> int:
+    """Enqueue the bounded-wait self-test (a wait that nothing satisfies)."""
+    return lib().vdn_selftest_bounded_wait(_ptr(workspace), int(limit_us), _stream(stream))
 
 
 def use_tc_params(p: VdnParams) -> bool:

@@ -186,6 +186,31 @@ def test_device_status_ok_and_range():
     assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"  # cleared
 
 
+def test_bounded_wait_expires_into_status():
+    """A wait that nothing satisfies ends at its limit with VDN_ERR_TIMEOUT in
+    the status word (no hang, no fault), and the context stays usable: the
+    same workspace then runs a forward to parity."""
+    import time
+    cfg = _edge_cfg(dict(T=10, N=32))
+    inp = make_inputs(cfg)
+    d = to_dev(inp)
+    p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"])
+    ws = vdn.alloc_workspace(p)
+    assert vdn.STATUS[vdn.selftest_bounded_wait(ws, 50)] == "VDN_ERR_INVALID_ARG"
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    assert vdn.STATUS[vdn.selftest_bounded_wait(ws, 20000)] == "VDN_OK"
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_ERR_TIMEOUT"
+    dt = time.perf_counter() - t0
+    assert 0.015 <= dt < 1.0, dt  # expired at its 20 ms limit, ended well before 2x + slack
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"  # cleared
+    out = _fwd(d, cfg, params=p, workspace=ws)
+    torch.cuda.synchronize()
+    assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    assert rel_err(out.double().cpu().numpy(), want) <= TOL_OUT["bf16"]
+
+
 # ----------------------------------------------------------------------------
 # full-size workloads, sampled rows
 # ----------------------------------------------------------------------------
