@@ -345,7 +345,9 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
     """The whole hybrid attention forward on the selected query rows.
 
     ``inp`` holds numpy (or torch CPU) arrays with the keys q, k, v, beta,
-    alpha (or None), text_k, text_v, W_soft, W_lin, gates.
+    alpha (or None), text_k, text_v, W_soft, W_lin, gates, and optionally
+    q_lin, k_lin, v_lin: the linear branch's own inputs (its feature map of
+    the projections); without them both branches read q, k, v.
     ``text_softmax``: video queries also attend all text tokens in the
     Softmax branch (one normaliser).
     Returns (out [B, R, D_out], o_s [B, R, H, d_v], o_l [B, R, H, d_v]).
@@ -356,7 +358,10 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
     o_s = softmax_branch(a["q"], a["k"], a["v"], T, N, chunk, radius, scale, rows,
                          text_k=a["text_k"] if text_softmax else None,
                          text_v=a["text_v"] if text_softmax else None)
-    o_l = linear_branch(a["q"], a["k"], a["v"], a["beta"], a["text_k"], a["text_v"],
+    ql = a["q_lin"] if a.get("q_lin") is not None else a["q"]
+    kl = a["k_lin"] if a.get("k_lin") is not None else a["k"]
+    vl = a["v_lin"] if a.get("v_lin") is not None else a["v"]
+    o_l = linear_branch(ql, kl, vl, a["beta"], a["text_k"], a["text_v"],
                         T, N, chunk, radius, a.get("alpha"), rows, text_full, beta_per_token)
     g = a["gates"]
     out = output_projection(o_s, o_l, g[0][:, rows], g[1][:, rows], a["W_soft"],

@@ -4,4 +4,5 @@ This package holds only the workload shapes and the random draws that both the
 CUDA path and the CPU oracle consume.  It contains none of the method's
 arithmetic.
 """
-from .inputs import CONFIGS, Config, make_inputs, sample_rows  # noqa: F401
+from .inputs import (CONFIGS, Config, grid_shape, make_inputs, make_prep_inputs,  # noqa: F401
+                     sample_rows)

@@ -160,3 +160,46 @@ def sample_rows(cfg: Config, per_frame: int = 4, extra_frac: float = 0.0,
         n_extra = int(extra_frac * cfg.L)
         rows += rng.choice(cfg.L, size=n_extra, replace=False).tolist()
     return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+def grid_shape(N: int) -> tuple:
+    """Spatial token grid (grid_h, grid_w) of a frame of N tokens: the factor
+    pair with grid_h <= grid_w closest to square (1536 -> 32 x 48,
+    576 -> 24 x 24, 256 -> 16 x 16)."""
+    h = int(np.floor(np.sqrt(N)))
+    while N % h:
+        h -= 1
+    return h, N // h
+
+
+def make_prep_inputs(cfg: Config, *, grid: Optional[tuple] = None, device: str = "cpu") -> dict:
+    """Raw inputs of the linear branch's feature map (VDA-Prep), drawn from a
+    second seeded generator (seed + 7919) so that ``make_inputs`` is unchanged:
+
+      1. q_raw, k_raw, v_raw [B, L, H, d] ~ N(0, 1)  (pretrained projections,
+         before any normalisation), rounded once to the workload dtype
+      2. wk_s [H*d, 3, 3] ~ N(0, 1) / 3,   wk_t [H*d, 5] ~ N(0, 1) / sqrt(5)
+      3. wv_s, wv_t likewise                (float32; random stand-ins for the
+         released depthwise spatial and five-tap temporal filters)
+
+    ``grid`` is the frame's (grid_h, grid_w); default ``grid_shape(N)``.
+    """
+    g = torch.Generator(device="cpu").manual_seed(cfg.seed + 7919)
+    B, H, d, L = cfg.B, cfg.H, cfg.d, cfg.L
+    dt = _TORCH_DTYPE[cfg.dtype]
+    gh, gw = grid_shape(cfg.N) if grid is None else grid
+    assert gh * gw == cfg.N
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+    out = {"grid_h": gh, "grid_w": gw}
+    for name in ("q_raw", "k_raw", "v_raw"):
+        out[name] = randn(B, L, H, d).to(dt)
+    out["wk_s"] = randn(H * d, 3, 3) / 3.0
+    out["wk_t"] = randn(H * d, 5) / np.sqrt(5.0)
+    out["wv_s"] = randn(H * d, 3, 3) / 3.0
+    out["wv_t"] = randn(H * d, 5) / np.sqrt(5.0)
+    if device != "cpu":
+        out = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in out.items()}
+    return out
