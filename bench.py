@@ -186,7 +186,10 @@ def base_line(args, cfg, value, ms_per_step, n_gpus):
                    "decay_gate": "U[0.9,1]" if getattr(args, "alpha", False) else "none",
                    "text_keys_in_softmax": bool(getattr(args, "text_softmax", False)),
                    "write_gate": "per token" if getattr(args, "beta_per_token", False)
-                                 else "per frame"},
+                                 else "per frame",
+                   "linear_feature_map": "VDA-Prep in the step (3x3 spatial + 5-tap temporal "
+                                         "conv, SiLU, L2; random filters)"
+                                         if getattr(args, "prep", False) else "inputs prepared"},
     }
 
 
@@ -243,11 +246,29 @@ def run_ours(args, cfg):
     ws = vdn.alloc_workspace(p)
     out = torch.empty(cfg.B, cfg.L, p.D_out, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    lin = None
+    if args.prep:  # raw projections -> VDA-Prep -> the linear branch's q, k, v
+        from synth import make_prep_inputs
+        pin = make_prep_inputs(cfg)
+        dp = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in pin.items()}
+        lin = tuple(torch.empty_like(dp[n]) for n in ("q_raw", "k_raw", "v_raw"))
+        pp = vdn.make_prep_params(cfg.B, cfg.H, cfg.T, pin["grid_h"], pin["grid_w"], cfg.d,
+                                  cfg.dtype)
+        prep_ws = torch.zeros(vdn.PREP_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    prep_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
 
-    def step(events=None):
+    def step(events=None, i=None):
+        if lin is not None:
+            if i is not None:
+                prep_ev[i][0].record(stream)
+            vdn.vda_prep(dp["q_raw"], dp["k_raw"], dp["v_raw"], dp["wk_s"], dp["wk_t"],
+                         dp["wv_s"], dp["wv_t"], cfg.T, pin["grid_h"], pin["grid_w"], out=lin,
+                         workspace=prep_ws, params=pp)
+            if i is not None:
+                prep_ev[i][1].record(stream)
         vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
                             d["W_soft"], d["W_lin"], d["gates"], cfg.T, alpha=d["alpha"],
-                            out=out, workspace=ws, params=p, events=events)
+                            out=out, workspace=ws, params=p, events=events, lin=lin)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -266,7 +287,7 @@ def run_ours(args, cfg):
     time.sleep(0.3)
     t_start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(evs[i], i)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -281,6 +302,13 @@ def run_ours(args, cfg):
     st = vdn.device_status(p, ws)
     if st != 0:
         raise RuntimeError(f"device status after timing: {vdn.STATUS[st]}")
+    prep_ms = None
+    if lin is not None:
+        prep_ms = sum(e[0].elapsed_time(e[1]) for e in prep_ev) / args.steps
+        st = vdn.device_status(None, prep_ws)
+        if st != 0:
+            raise RuntimeError(f"device status of VDA-Prep: {vdn.STATUS[st]}")
+        del dp, lin
 
     ms_per_step = elapsed_ms / args.steps
     tokens = cfg.B * cfg.L
@@ -340,11 +368,24 @@ def run_ours(args, cfg):
             "peak_tflops": pk["tc"], "peak_hbm_gbs": pk["hbm"], "peaks": pk["src"] + " (burst)",
         }
         line["stages_ms"] = dict(zip(vdn.STAGE_NAMES, [round(x, 4) for x in stage_ms]))
-        line["gpu_launches"] = args.steps * (8 if vdn.use_tc_params(p) else 6)
+        line["gpu_launches"] = args.steps * ((8 if vdn.use_tc_params(p) else 6) +
+                                             (2 if prep_ms is not None else 0))
+        if prep_ms is not None:
+            es = 2 if cfg.dtype == "bf16" else 4
+            prep_bytes = 6 * cfg.B * cfg.L * cfg.H * cfg.d * es  # read q, k, v; write 3
+            line["stages_ms"]["prep"] = round(prep_ms, 4)
+            line["prep_roofline"] = {
+                "bound": "hbm", "kernel": "prep_conv_kernel + prep_l2_kernel (VDA-Prep)",
+                "achieved": prep_bytes / (prep_ms / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": prep_bytes / (prep_ms / 1e3) / 1e9 / pk["hbm"], "traffic": None,
+                "algorithmic_bytes_per_launch": prep_bytes, "ms_per_launch": prep_ms,
+                "peak_kind": f"{pk['src']} HBM copy"}
         line["clocks"] = clocks
         line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                        "api": "HostPipeline (pinned host buffers, 3 streams, 2 slots)"}
+        if args.prep:
+            line["e2e"]["note"] = "the forward on prepared inputs; VDA-Prep is not in this leg"
         if world == 1 and not args.no_cpu_baseline:
             rows = oracle_sample(cfg, inp)
             secs = time_oracle(cfg, inp, rows)
@@ -372,6 +413,8 @@ def main():
                     help="video queries also attend all text tokens in the Softmax branch")
     ap.add_argument("--beta-per-token", action="store_true",
                     help="one write gate per token instead of per frame")
+    ap.add_argument("--prep", action="store_true",
+                    help="time VDA-Prep (linear-branch feature map of raw q, k, v) in every step")
     ap.add_argument("--alpha", action="store_true",
                     help="channel-wise decay gate alpha ~ U[0.9, 1] instead of none")
     args = ap.parse_args()

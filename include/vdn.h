@@ -175,6 +175,73 @@ VDN_API vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params *p, const void *q
                                       size_t workspace_bytes, vdn_stream_t stream,
                                       const vdn_stage_events *ev);
 
+/* vdn_hybrid_attn_fwd_staged with the linear branch reading its own inputs:
+ * the method feeds the linear branch from the same projections through its
+ * own feature map (vdn_vda_prep), while the Softmax branch keeps q, k, v.
+ *  - q, k, v: Softmax branch inputs, as for vdn_hybrid_attn_fwd.
+ *  - q_lin, k_lin, v_lin: [B, L, H, d] dtype params.dtype, the linear branch's
+ *    queries (readout), keys and values (frame statistics).  Passing q, k, v
+ *    again gives exactly vdn_hybrid_attn_fwd_staged.
+ *  - text_k, text_v serve both branches; every other argument, the workspace
+ *    size and the events as vdn_hybrid_attn_fwd_staged. */
+VDN_API vdn_status vdn_hybrid_attn_fwd_split(const vdn_params *p, const void *q, const void *k,
+                                     const void *v, const void *q_lin, const void *k_lin,
+                                     const void *v_lin, const float *beta, const float *alpha,
+                                     const void *text_k, const void *text_v,
+                                     const void *W_o_soft, const void *W_o_lin,
+                                     const void *gates, void *out, void *workspace,
+                                     size_t workspace_bytes, vdn_stream_t stream,
+                                     const vdn_stage_events *ev);
+
+/* ---- VDA-Prep: the linear branch's feature map ----------------------------
+ * "Video DeltaNet" method (the linear branch applies its own feature map to
+ * the pretrained projections: a separable short convolution of K and V -- a
+ * depthwise spatial filter and a five-tap temporal filter -- then SiLU, and L2
+ * normalisation of Q and K) and implementation ("Fused VDA kernels",
+ * VDA-Prep).  Computed, in FP32:
+ *   k_l = L2(SiLU(conv_t(conv_s(k)))),  v_l = SiLU(conv_t(conv_s(v))),
+ *   q_l = L2(q),   L2(x) = x / sqrt(sum_d x^2 + l2_eps) per (token, head).
+ * conv_s: depthwise 3x3 cross-correlation over the frame's row-major
+ * grid_h x grid_w token grid (token n = y * grid_w + x), zero padding;
+ * conv_t: depthwise 5 taps over frames t-2 .. t+2, zero padding at the clip
+ * ends.  Video tokens only (text tokens have no grid).  Outputs are rounded
+ * once to dtype. */
+typedef struct vdn_prep_params {
+  int B, H, T;          /* batch, heads, latent frames */
+  int grid_h, grid_w;   /* tokens per frame N = grid_h * grid_w */
+  int d;                /* head dim: 32, 64 or 128 */
+  int spatial_taps;     /* 3 (the only size served) */
+  int temporal_taps;    /* 5 (the only size served) */
+  vdn_dtype dtype;      /* of q, k, v and of the outputs */
+  float l2_eps;         /* default 1e-6 */
+} vdn_prep_params;
+
+/* Workspace of vdn_vda_prep: its device status word. */
+#define VDN_PREP_WORKSPACE_BYTES 256u
+
+/* Fills defaults (3x3 spatial, 5 temporal taps, l2_eps 1e-6) and validates. */
+VDN_API vdn_status vdn_prep_params_init(vdn_prep_params *p, int B, int H, int T, int grid_h,
+                                        int grid_w, int d, vdn_dtype dtype);
+
+/*  - q, k, v: [B, T*grid_h*grid_w, H, d] dtype, device.  Either group may be
+ *    skipped: q = q_out = NULL skips Q; k, v, k_out, v_out and the four
+ *    filters all NULL skips K/V.
+ *  - wk_s, wv_s: float32 [H*d][3][3] spatial filters of K and V (channel
+ *    c = h*d + i, then filter row, then column); wk_t, wv_t: float32
+ *    [H*d][5] temporal filters (tap j weighs frame t + j - 2).
+ *  - q_out, k_out, v_out: [B, T*grid_h*grid_w, H, d] dtype.  k_out and v_out
+ *    must not overlap k, v or each other (VDN_ERR_INVALID_ARG); q_out may be q.
+ *  - workspace: >= VDN_PREP_WORKSPACE_BYTES bytes of device memory, 256-byte
+ *    aligned; holds the device status word (read it with
+ *    vdn_device_status(NULL, workspace, stream)).
+ *  - Other conventions as the forward: 16-byte aligned pointers, validation
+ *    before any launch, asynchronous on `stream`. */
+VDN_API vdn_status vdn_vda_prep(const vdn_prep_params *p, const void *q, const void *k,
+                                const void *v, const float *wk_s, const float *wk_t,
+                                const float *wv_s, const float *wv_t, void *q_out, void *k_out,
+                                void *v_out, void *workspace, size_t workspace_bytes,
+                                vdn_stream_t stream);
+
 /* The two branch readouts before gating and projection, float32
  * [B, L, H, d_v]: o_soft = Softmax branch, o_lin = linear branch before its
  * RMS norm.  Either output pointer may be NULL to skip that branch. */
@@ -223,7 +290,8 @@ VDN_API vdn_status vdn_vda_boundary_states_noalloc(const vdn_params *p, const vo
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * the last compute call on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
- * VDN_ERR_RANGE).  `workspace` must be the one passed to that call. */
+ * VDN_ERR_RANGE).  `workspace` must be the one passed to that call.  `p` may
+ * be NULL (it is only validated when given). */
 VDN_API vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_stream_t stream);
 
 /* Self-test of failure detection, without a fault or a hang.

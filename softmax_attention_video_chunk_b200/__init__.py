@@ -49,6 +49,17 @@ class VdnParams(ctypes.Structure):
     ]
 
 
+class VdnPrepParams(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+        ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("d", ctypes.c_int),
+        ("spatial_taps", ctypes.c_int), ("temporal_taps", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("l2_eps", ctypes.c_float),
+    ]
+
+
+PREP_WORKSPACE_BYTES = 256
+
 _lib = None
 _P = ctypes.c_void_p
 
@@ -83,6 +94,14 @@ def lib() -> ctypes.CDLL:
         L.vdn_vda_boundary_states_noalloc.argtypes = [PP] + [_P] * 8 + [_P]
         L.vdn_device_status.restype = ctypes.c_int
         L.vdn_device_status.argtypes = [PP, _P, _P]
+        L.vdn_hybrid_attn_fwd_split.restype = ctypes.c_int
+        L.vdn_hybrid_attn_fwd_split.argtypes = ([PP] + [_P] * 15 + [ctypes.c_size_t, _P] +
+                                                [ctypes.POINTER(VdnStageEvents)])
+        PPP = ctypes.POINTER(VdnPrepParams)
+        L.vdn_prep_params_init.restype = ctypes.c_int
+        L.vdn_prep_params_init.argtypes = [PPP] + [ctypes.c_int] * 7
+        L.vdn_vda_prep.restype = ctypes.c_int
+        L.vdn_vda_prep.argtypes = [PPP] + [_P] * 11 + [ctypes.c_size_t, _P]
         L.vdn_selftest_bounded_wait.restype = ctypes.c_int
         L.vdn_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint, _P]
         _lib = L
@@ -162,11 +181,14 @@ def alloc_workspace(p: VdnParams, device="cuda"):
 
 
 def hybrid_attn_fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, *, alpha=None,
-                    out=None, workspace=None, stream=None, params=None, events=None, **kw):
+                    out=None, workspace=None, stream=None, params=None, events=None, lin=None,
+                    **kw):
     """out [B, L, D_out] = VDN hybrid attention forward (all steps in libvdn).
 
     ``events``: optional list of N_STAGES + 1 torch.cuda.Event(enable_timing=True)
-    recorded at the stage boundaries (see vdn_hybrid_attn_fwd_staged)."""
+    recorded at the stage boundaries (see vdn_hybrid_attn_fwd_staged).
+    ``lin``: optional (q_lin, k_lin, v_lin), the linear branch's own inputs
+    (vdn_hybrid_attn_fwd_split); by default both branches read q, k, v."""
     import torch
     p = params or params_for(q, v, text_k, T, W_soft, **kw)
     if out is None:
@@ -183,12 +205,53 @@ def hybrid_attn_fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, *, a
                 e.record(torch.cuda.current_stream() if stream is None else stream)
             ev.events[i] = e.cuda_event
         ev = ctypes.byref(ev)
-    rc = lib().vdn_hybrid_attn_fwd_staged(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
-                                          _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(W_soft),
-                                          _ptr(W_lin), _ptr(gates), _ptr(out), _ptr(ws),
-                                          ws.numel(), _stream(stream), ev)
+    if lin is None:
+        rc = lib().vdn_hybrid_attn_fwd_staged(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(beta), _ptr(alpha), _ptr(text_k),
+                                              _ptr(text_v), _ptr(W_soft), _ptr(W_lin),
+                                              _ptr(gates), _ptr(out), _ptr(ws), ws.numel(),
+                                              _stream(stream), ev)
+    else:
+        ql, kl, vl = lin
+        rc = lib().vdn_hybrid_attn_fwd_split(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(ql), _ptr(kl), _ptr(vl), _ptr(beta),
+                                             _ptr(alpha), _ptr(text_k), _ptr(text_v),
+                                             _ptr(W_soft), _ptr(W_lin), _ptr(gates), _ptr(out),
+                                             _ptr(ws), ws.numel(), _stream(stream), ev)
     if rc != 0:
         raise VdnError(rc, "vdn_hybrid_attn_fwd")
+    return out
+
+
+def make_prep_params(B, H, T, grid_h, grid_w, d, dtype="bf16", l2_eps=1e-6) -> VdnPrepParams:
+    p = VdnPrepParams()
+    rc = lib().vdn_prep_params_init(ctypes.byref(p), B, H, T, grid_h, grid_w, d,
+                                    {"f32": VDN_F32, "bf16": VDN_BF16}[dtype])
+    if rc != 0:
+        raise VdnError(rc, "vdn_prep_params_init")
+    p.l2_eps = l2_eps
+    return p
+
+
+def vda_prep(q, k, v, wk_s, wk_t, wv_s, wv_t, T, grid_h, grid_w, *, l2_eps=1e-6, out=None,
+             workspace=None, stream=None, params=None):
+    """(q_l, k_l, v_l) = VDA-Prep of the raw projections (see vdn_vda_prep):
+    q_l = L2(q), k_l = L2(SiLU(conv(k))), v_l = SiLU(conv(v)).  Inputs
+    [B, T*grid_h*grid_w, H, d]; filters float32 [H*d, 3, 3] and [H*d, 5].
+    Pass q = None to skip Q, or k = v = None (and the filters) to skip K/V."""
+    import torch
+    x = k if k is not None else q
+    B, L, H, d = x.shape
+    p = params or make_prep_params(B, H, T, grid_h, grid_w, d, _dtype_name(x), l2_eps)
+    if out is None:
+        out = tuple(None if t is None else torch.empty_like(t) for t in (q, k, v))
+    ws = (torch.empty(PREP_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+          if workspace is None else workspace)
+    rc = lib().vdn_vda_prep(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(wk_s), _ptr(wk_t),
+                            _ptr(wv_s), _ptr(wv_t), _ptr(out[0]), _ptr(out[1]), _ptr(out[2]),
+                            _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_vda_prep")
     return out
 
 
@@ -280,9 +343,11 @@ def vda_boundary_states_noalloc(k, v, beta, text_k, text_v, T, *, alpha=None, st
     return F, G
 
 
-def device_status(p: VdnParams, workspace, stream=None) -> int:
-    """Synchronise and return (and clear) the device status of the last call."""
-    return lib().vdn_device_status(ctypes.byref(p), _ptr(workspace), _stream(stream))
+def device_status(p: Optional[VdnParams], workspace, stream=None) -> int:
+    """Synchronise and return (and clear) the device status of the last call
+    (``p`` may be None, e.g. for the VDA-Prep workspace)."""
+    return lib().vdn_device_status(None if p is None else ctypes.byref(p), _ptr(workspace),
+                                   _stream(stream))
 
 
 def selftest_bounded_wait(workspace, limit_us: int, stream=None) -> int:

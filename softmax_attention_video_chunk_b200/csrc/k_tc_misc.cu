@@ -45,8 +45,9 @@ static EncodeTiledFn encode_fn() {
 }
 
 // Tiled map with 128-byte swizzle; dims/box innermost first; strides of dims 1..
-bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
-               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+static bool make_tmap_sw(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                         const uint64_t* dims, const uint64_t* strides_bytes,
+                         const uint32_t* box, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t d[5], s[4];
@@ -58,9 +59,21 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* b
     if (i + 1 < rank) s[i] = strides_bytes[i];
   }
   const CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, s, bx, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 128-byte swizzled boxes (the tensor-core operand tiles).
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap_sw(map, dt, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Dense (unswizzled) boxes, laid out in shared memory in row-major box order.
+bool make_tmap_plain(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                     const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_tmap_sw(map, dt, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // --------------------------------------------------------------------------
@@ -378,7 +391,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
-static int sm_count() {
+int sm_count() {
   static int cached[128] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;

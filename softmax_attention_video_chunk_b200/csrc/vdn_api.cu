@@ -102,6 +102,19 @@ vdn_status boundary_states_impl(const vdn_params* p, const void* k, const void* 
                                 const void* text_v, float* F, float* G, void* workspace,
                                 vdn_stream_t stream);
 
+static vdn_status validate_prep(const vdn_prep_params* p) {
+  if (p == nullptr) return VDN_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->T < 1 || p->grid_h < 1 || p->grid_w < 1) return VDN_ERR_SHAPE;
+  if (p->d != 32 && p->d != 64 && p->d != 128) return VDN_ERR_UNSUPPORTED;
+  if (p->spatial_taps != 3 || p->temporal_taps != 5) return VDN_ERR_UNSUPPORTED;
+  if (p->dtype != VDN_F32 && p->dtype != VDN_BF16) return VDN_ERR_DTYPE;
+  if (!(p->l2_eps >= 0.f) || p->l2_eps > 1.f) return VDN_ERR_INVALID_ARG;
+  // the TMA frame coordinate and the grid extents are 32-bit
+  if ((long long)p->B * p->T > (1ll << 30) || (long long)p->grid_h * p->grid_w > (1ll << 30))
+    return VDN_ERR_SHAPE;
+  return VDN_OK;
+}
+
 static vdn_status check_ws(const vdn_params* p, const void* ws, size_t ws_bytes) {
   const WsLayout w = layout(*p);
   if (ws == nullptr || ws_bytes < w.total) return VDN_ERR_WORKSPACE;
@@ -281,15 +294,22 @@ vdn_status vdn_hybrid_attn_branches(const vdn_params* p, const void* q, const vo
   return VDN_OK;
 }
 
-vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const void* k,
-                                      const void* v, const float* beta, const float* alpha,
-                                      const void* text_k, const void* text_v,
-                                      const void* W_o_soft, const void* W_o_lin,
-                                      const void* gates, void* out, void* workspace,
-                                      size_t workspace_bytes, vdn_stream_t stream,
-                                      const vdn_stage_events* ev) {
+}  // extern "C"
+
+namespace vdn {
+// The forward with the linear branch reading its own q_l, k_l, v_l (equal to
+// q, k, v unless the caller passes the linear feature map's outputs).
+static vdn_status fwd_impl(const vdn_params* p, const void* q, const void* k, const void* v,
+                           const void* q_l, const void* k_l, const void* v_l, const float* beta,
+                           const float* alpha, const void* text_k, const void* text_v,
+                           const void* W_o_soft, const void* W_o_lin, const void* gates,
+                           void* out, void* workspace, size_t workspace_bytes,
+                           vdn_stream_t stream, const vdn_stage_events* ev) {
   VDN_TRY(validate_params(p));
   VDN_TRY(common_inputs(p, q, k, v, beta, alpha, text_k, text_v, true));
+  VDN_TRY(check_ptr(q_l, true));
+  VDN_TRY(check_ptr(k_l, true));
+  VDN_TRY(check_ptr(v_l, true));
   VDN_TRY(check_ptr(W_o_soft, true));
   VDN_TRY(check_ptr(W_o_lin, true));
   VDN_TRY(check_ptr(gates, true));
@@ -306,11 +326,12 @@ vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const 
   const WsLayout w = layout(*p);
   VDN_CUDA(mark(0));
   VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
-  VdaArgs va = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+  VdaArgs va = vda_args(p, k_l, v_l, beta, alpha, text_k, text_v, ws);
   AttnArgs aa = attn_args(p, q, k, v, text_k, text_v);
   if (use_tc(*p)) {
     TcAttnArgs t = tc_attn_args(*p, aa, ws + w.vt, (int*)(ws + w.status));
     TcFwdArgs f = tc_fwd_args(*p, va, t, W_o_soft, W_o_lin, gates, out, ws + w.wt, ws + w.x);
+    f.q = q_l;  // the readout's queries
     VDN_CUDA(launch_vda_states(va, st));
     VDN_CUDA(mark(1));
     VDN_CUDA(launch_convert_v(t, st));
@@ -331,7 +352,7 @@ vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const 
   VDN_CUDA(mark(2));
   VDN_CUDA(launch_attn_simt(aa, o_s, st));
   VDN_CUDA(mark(3));
-  VDN_CUDA(launch_vda_readout_simt(va, q, o_l, st));
+  VDN_CUDA(launch_vda_readout_simt(va, q_l, o_l, st));
   VDN_CUDA(mark(4));
   ProjArgs pa;
   pa.B = p->B; pa.H = p->H; pa.L = p->T * p->N; pa.D = p->d_k; pa.D_out = p->D_out;
@@ -343,6 +364,33 @@ vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const 
   return VDN_OK;
 }
 
+}  // namespace vdn
+
+extern "C" {
+
+vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params* p, const void* q, const void* k,
+                                      const void* v, const float* beta, const float* alpha,
+                                      const void* text_k, const void* text_v,
+                                      const void* W_o_soft, const void* W_o_lin,
+                                      const void* gates, void* out, void* workspace,
+                                      size_t workspace_bytes, vdn_stream_t stream,
+                                      const vdn_stage_events* ev) {
+  return fwd_impl(p, q, k, v, q, k, v, beta, alpha, text_k, text_v, W_o_soft, W_o_lin, gates,
+                  out, workspace, workspace_bytes, stream, ev);
+}
+
+vdn_status vdn_hybrid_attn_fwd_split(const vdn_params* p, const void* q, const void* k,
+                                     const void* v, const void* q_lin, const void* k_lin,
+                                     const void* v_lin, const float* beta, const float* alpha,
+                                     const void* text_k, const void* text_v,
+                                     const void* W_o_soft, const void* W_o_lin,
+                                     const void* gates, void* out, void* workspace,
+                                     size_t workspace_bytes, vdn_stream_t stream,
+                                     const vdn_stage_events* ev) {
+  return fwd_impl(p, q, k, v, q_lin, k_lin, v_lin, beta, alpha, text_k, text_v, W_o_soft,
+                  W_o_lin, gates, out, workspace, workspace_bytes, stream, ev);
+}
+
 vdn_status vdn_hybrid_attn_fwd(const vdn_params* p, const void* q, const void* k, const void* v,
                                const float* beta, const float* alpha, const void* text_k,
                                const void* text_v, const void* W_o_soft, const void* W_o_lin,
@@ -352,8 +400,63 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_params* p, const void* q, const void* k
                                     gates, out, workspace, workspace_bytes, stream, nullptr);
 }
 
+vdn_status vdn_prep_params_init(vdn_prep_params* p, int B, int H, int T, int grid_h,
+                                int grid_w, int d, vdn_dtype dtype) {
+  if (p == nullptr) return VDN_ERR_INVALID_ARG;
+  memset(p, 0, sizeof(*p));
+  p->B = B; p->H = H; p->T = T; p->grid_h = grid_h; p->grid_w = grid_w; p->d = d;
+  p->spatial_taps = 3; p->temporal_taps = 5; p->dtype = dtype; p->l2_eps = 1e-6f;
+  return validate_prep(p);
+}
+
+vdn_status vdn_vda_prep(const vdn_prep_params* p, const void* q, const void* k, const void* v,
+                        const float* wk_s, const float* wk_t, const float* wv_s,
+                        const float* wv_t, void* q_out, void* k_out, void* v_out,
+                        void* workspace, size_t workspace_bytes, vdn_stream_t stream) {
+  VDN_TRY(validate_prep(p));
+  const bool has_q = q != nullptr || q_out != nullptr;
+  const bool has_kv = k != nullptr || v != nullptr || k_out != nullptr || v_out != nullptr ||
+                      wk_s != nullptr || wk_t != nullptr || wv_s != nullptr || wv_t != nullptr;
+  if (!has_q && !has_kv) return VDN_ERR_INVALID_ARG;
+  if (has_q) {
+    VDN_TRY(check_ptr(q, true));
+    VDN_TRY(check_ptr(q_out, true));
+  }
+  if (has_kv) {
+    const void* need[8] = {k, v, k_out, v_out, wk_s, wk_t, wv_s, wv_t};
+    for (const void* ptr : need) VDN_TRY(check_ptr(ptr, true));
+    // the convolution reads neighbours: no output may overlap an input
+    const size_t n = (size_t)p->B * p->T * p->grid_h * p->grid_w * p->H * p->d *
+                     (p->dtype == VDN_BF16 ? 2 : 4);
+    auto overlap = [n](const void* a, const void* b) {
+      const char *x = (const char*)a, *y = (const char*)b;
+      return x < y + n && y < x + n;
+    };
+    const void* outs[2] = {k_out, v_out};
+    const void* ins[2] = {k, v};
+    for (const void* o : outs)
+      for (const void* i : ins)
+        if (overlap(o, i)) return VDN_ERR_INVALID_ARG;
+    if (overlap(k_out, v_out)) return VDN_ERR_INVALID_ARG;
+  }
+  if (workspace == nullptr || workspace_bytes < VDN_PREP_WORKSPACE_BYTES)
+    return VDN_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255u) != 0) return VDN_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaMemsetAsync(workspace, 0, sizeof(int), st));
+  PrepArgs a;
+  a.B = p->B; a.H = p->H; a.T = p->T; a.gh = p->grid_h; a.gw = p->grid_w; a.D = p->d;
+  a.bf16 = p->dtype == VDN_BF16; a.eps = p->l2_eps;
+  a.q = has_q ? q : nullptr; a.q_out = has_q ? q_out : nullptr;
+  a.k = has_kv ? k : nullptr; a.v = v; a.k_out = k_out; a.v_out = v_out;
+  a.wk_s = wk_s; a.wk_t = wk_t; a.wv_s = wv_s; a.wv_t = wv_t;
+  a.status = (int*)workspace;
+  VDN_CUDA(launch_prep(a, st));
+  return VDN_OK;
+}
+
 vdn_status vdn_device_status(const vdn_params* p, void* workspace, vdn_stream_t stream) {
-  VDN_TRY(validate_params(p));
+  if (p != nullptr) VDN_TRY(validate_params(p));
   if (workspace == nullptr) return VDN_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   VDN_CUDA(cudaStreamSynchronize(st));

@@ -49,4 +49,16 @@ struct ProjArgs {
 };
 cudaError_t launch_proj_simt(const ProjArgs& a, cudaStream_t st);
 
+// VDA-Prep (linear-branch feature map); k == nullptr skips K/V, q == nullptr Q.
+struct PrepArgs {
+  int B, H, T, gh, gw, D;
+  bool bf16;
+  float eps;
+  const void *q, *k, *v;                         // [B, T*gh*gw, H, D]
+  const float *wk_s, *wk_t, *wv_s, *wv_t;        // [H*D][9], [H*D][5]
+  void *q_out, *k_out, *v_out;                   // [B, T*gh*gw, H, D]
+  int* status;
+};
+cudaError_t launch_prep(const PrepArgs& a, cudaStream_t st);
+
 }  // namespace vdn

@@ -121,3 +121,57 @@ def test_branches_and_states_validate():
                                    0x6008, None, 0x7f0000000000, need, None)
     assert vdn.STATUS[rc] == "VDN_ERR_ALIGNMENT"
     assert vdn.STATUS[L.vdn_device_status(ctypes.byref(p), None, None)] == "VDN_ERR_WORKSPACE"
+
+
+def _prep_call(p, ptrs, ws=0x7000, ws_bytes=256):
+    L = vdn.lib()
+    return vdn.STATUS[L.vdn_vda_prep(ctypes.byref(p), *[ctypes.c_void_p(x) for x in ptrs],
+                                     ctypes.c_void_p(ws), ws_bytes, None)]
+
+
+def test_prep_params_defaults_and_validation():
+    p = vdn.make_prep_params(1, 24, 75, 32, 48, 128, "bf16")
+    assert (p.spatial_taps, p.temporal_taps) == (3, 5) and abs(p.l2_eps - 1e-6) < 1e-12
+    L = vdn.lib()
+    for field, value, code in [("d", 96, "VDN_ERR_UNSUPPORTED"), ("spatial_taps", 5, "VDN_ERR_UNSUPPORTED"),
+                               ("temporal_taps", 3, "VDN_ERR_UNSUPPORTED"), ("grid_w", 0, "VDN_ERR_SHAPE"),
+                               ("T", 0, "VDN_ERR_SHAPE"), ("dtype", 4, "VDN_ERR_DTYPE"),
+                               ("l2_eps", -1.0, "VDN_ERR_INVALID_ARG")]:
+        q = vdn.make_prep_params(1, 2, 4, 3, 5, 64, "bf16")
+        setattr(q, field, value)
+        ptrs = [0x1000 * (i + 1) for i in range(10)]
+        assert _prep_call(q, ptrs) == code, field
+
+
+def test_prep_rejects_bad_arguments_before_launch():
+    p = vdn.make_prep_params(1, 2, 4, 3, 5, 64, "bf16")
+    n = 4 * 15 * 2 * 64 * 2  # bytes of one tensor
+    # q k v wk_s wk_t wv_s wv_t q_out k_out v_out
+    base = [0x100000 * (i + 1) for i in range(10)]
+    assert _prep_call(p, [0] * 10) == "VDN_ERR_INVALID_ARG"  # nothing to do
+    bad = list(base)
+    bad[1] = 0  # k missing while v present
+    assert _prep_call(p, bad) == "VDN_ERR_INVALID_ARG"
+    bad = list(base)
+    bad[3] = 0x400008  # misaligned filter
+    assert _prep_call(p, bad) == "VDN_ERR_ALIGNMENT"
+    bad = list(base)
+    bad[8] = base[2] + n // 2  # k_out overlaps v
+    assert _prep_call(p, bad) == "VDN_ERR_INVALID_ARG"
+    bad = list(base)
+    bad[9] = bad[8]  # k_out == v_out
+    assert _prep_call(p, bad) == "VDN_ERR_INVALID_ARG"
+    assert _prep_call(p, [base[0]] + [0] * 9) == "VDN_ERR_INVALID_ARG"  # q without q_out
+    assert _prep_call(p, base, ws=0) == "VDN_ERR_WORKSPACE"
+    assert _prep_call(p, base, ws_bytes=255) == "VDN_ERR_WORKSPACE"
+    assert _prep_call(p, base, ws=0x7010) == "VDN_ERR_ALIGNMENT"
+
+
+def test_split_forward_requires_linear_inputs():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    L = vdn.lib()
+    ptr = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(14)]
+    ptr[3] = ctypes.c_void_p(0)  # q_lin missing
+    rc = L.vdn_hybrid_attn_fwd_split(ctypes.byref(p), *ptr, ctypes.c_void_p(0x80000),
+                                     1 << 40, None, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"
