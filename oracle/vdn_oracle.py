@@ -193,11 +193,23 @@ def vda_solve(A, W, S_prev, alpha=None):
     return np.linalg.solve(np.eye(dk) + A, S_tilde + W)
 
 
-def vda_update(S_prev, K, V, beta, alpha=None):
+def frozen_solve(A, W, S_prev, alpha=None):
+    """Frozen-state (SANA-WM) batched frame update from the same statistics,
+    the comparison rule of the Video Delta Attention section: every token's
+    correction is evaluated at the same decayed state S~ = Diag(alpha) S_prev,
+    S = S~ + sum_i beta_i k_i (v_i - S~^T k_i)^T = (I - A) S~ + W.  (The
+    pages also scale SANA-WM's keys by a frame-size factor whose symbol was
+    lost; keys are taken as given, so a caller applies any such factor.)"""
+    S_tilde = decay(np.asarray(S_prev, F64), alpha)
+    return S_tilde - A @ S_tilde + W
+
+
+def vda_update(S_prev, K, V, beta, alpha=None, frozen=False):
     """One Video Delta Attention frame update from the frame's keys K [n, d_k],
-    values V [n, d_v] and write gate beta."""
+    values V [n, d_v] and write gate beta (``frozen``: the frozen-state rule
+    instead)."""
     A, W = frame_stats(K, V, beta)
-    return vda_solve(A, W, S_prev, alpha)
+    return (frozen_solve if frozen else vda_solve)(A, W, S_prev, alpha)
 
 
 def decay(S, alpha):
@@ -207,13 +219,13 @@ def decay(S, alpha):
     return np.asarray(alpha, F64)[:, None] * S
 
 
-def text_state(text_k, text_v, beta0):
+def text_state(text_k, text_v, beta0, frozen=False):
     """S_text: the text tokens as one leading virtual frame, updated from the
     zero state (method, the text-aware initial state of both scans)."""
     text_k = np.asarray(text_k, F64)
     text_v = np.asarray(text_v, F64)
     S0 = np.zeros((text_k.shape[1], text_v.shape[1]), F64)
-    return vda_update(S0, text_k, text_v, beta0)
+    return vda_update(S0, text_k, text_v, beta0, frozen=frozen)
 
 
 def _frame_beta(beta_bh, t, N, n_text, per_token):
@@ -246,25 +258,27 @@ class _FrameStats:
         return self.cache[t]
 
 
-def _scan_outside_window(stats, alpha_bh, init, T, lo, hi):
+def _scan_outside_window(stats, alpha_bh, init, T, lo, hi, frozen=False):
     """Forward state after frames [0, lo) and reverse state after frames
     [hi, T), each run frame by frame from ``init``; anchors decay only (R4)."""
     A = anchor_frames(T)
+    solve = frozen_solve if frozen else vda_solve
 
     def al(t):
         return None if alpha_bh is None else alpha_bh[t]
 
     Sf = init.copy()
     for t in range(0, lo):
-        Sf = decay(Sf, al(t)) if t in A else vda_solve(*stats(t), Sf, al(t))
+        Sf = decay(Sf, al(t)) if t in A else solve(*stats(t), Sf, al(t))
     Sr = init.copy()
     for t in range(T - 1, hi - 1, -1):
-        Sr = decay(Sr, al(t)) if t in A else vda_solve(*stats(t), Sr, al(t))
+        Sr = decay(Sr, al(t)) if t in A else solve(*stats(t), Sr, al(t))
     return Sf, Sr
 
 
 def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
-                  alpha=None, rows=None, text_full=False, beta_per_token=False):
+                  alpha=None, rows=None, text_full=False, beta_per_token=False,
+                  frozen=False):
     """Linear (VDA) branch readout o_l = q^T S_f + q^T S_r for every (b, h)
     (method: the distant-context output adds the forward and reverse readouts).
 
@@ -274,7 +288,8 @@ def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
     query frame then bridges them with decay only across the window frames
     between the window edge and itself, inclusive (R6).  Anchor queries read
     1/2 S_text from each direction (R3).  The scan starts from 1/2 S_text
-    (R5; ``text_full`` starts from S_text).
+    (R5; ``text_full`` starts from S_text).  ``frozen``: every frame update
+    (text frame included) follows the frozen-state rule (frozen_solve).
     Returns [B, R, H, d_v] (before RMS norm and gate).
     """
     q = np.asarray(q, F64)
@@ -293,7 +308,7 @@ def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
     for b in range(B):
         for h in range(H):
             S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :],
-                                _text_beta(beta[b, h], nt, beta_per_token))
+                                _text_beta(beta[b, h], nt, beta_per_token), frozen)
             init = S_text if text_full else 0.5 * S_text
             al = None if alpha is None else np.asarray(alpha, F64)[b, h]
             stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N, nt, beta_per_token)
@@ -307,7 +322,8 @@ def linear_branch(q, k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
                     lo, hi = win[0], win[-1] + 1
                     c = t_q // chunk
                     if c not in per_chunk:
-                        per_chunk[c] = _scan_outside_window(stats, al, init, T, lo, hi)
+                        per_chunk[c] = _scan_outside_window(stats, al, init, T, lo, hi,
+                                                            frozen)
                     Sf, Sr = per_chunk[c]
                     for t in range(lo, t_q + 1):          # forward bridge
                         Sf = decay(Sf, None if al is None else al[t])
@@ -341,7 +357,8 @@ def output_projection(o_s, o_l, g_s, g_l, W_soft, W_lin, eps=1e-6):
 
 
 def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
-                   rows=None, text_full=False, text_softmax=False, beta_per_token=False):
+                   rows=None, text_full=False, text_softmax=False, beta_per_token=False,
+                   frozen=False):
     """The whole hybrid attention forward on the selected query rows.
 
     ``inp`` holds numpy (or torch CPU) arrays with the keys q, k, v, beta,
@@ -362,7 +379,8 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
     kl = a["k_lin"] if a.get("k_lin") is not None else a["k"]
     vl = a["v_lin"] if a.get("v_lin") is not None else a["v"]
     o_l = linear_branch(ql, kl, vl, a["beta"], a["text_k"], a["text_v"],
-                        T, N, chunk, radius, a.get("alpha"), rows, text_full, beta_per_token)
+                        T, N, chunk, radius, a.get("alpha"), rows, text_full, beta_per_token,
+                        frozen)
     g = a["gates"]
     out = output_projection(o_s, o_l, g[0][:, rows], g[1][:, rows], a["W_soft"],
                             a["W_lin"], eps)
@@ -370,7 +388,7 @@ def hybrid_forward(inp: dict, T, N, chunk=5, radius=1, scale=None, eps=1e-6,
 
 
 def boundary_states(k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
-                    alpha=None, text_full=False, beta_per_token=False):
+                    alpha=None, text_full=False, beta_per_token=False, frozen=False):
     """For every (b, h) and query chunk c, the forward and reverse states that
     a query of chunk c reads before its bridge: forward = after all frames
     before the window, reverse = after all frames after the window, each
@@ -390,14 +408,15 @@ def boundary_states(k, v, beta, text_k, text_v, T, N, chunk=5, radius=1,
     for b in range(B):
         for h in range(H):
             S_text = text_state(text_k[b, :, h, :], text_v[b, :, h, :],
-                                _text_beta(beta[b, h], nt, beta_per_token))
+                                _text_beta(beta[b, h], nt, beta_per_token), frozen)
             init = S_text if text_full else 0.5 * S_text
             al = None if alpha is None else np.asarray(_to_np(alpha), F64)[b, h]
             stats = _FrameStats(k[b, :, h, :], v[b, :, h, :], beta[b, h], N, nt, beta_per_token)
             for c in range(nc):
                 lo = max(0, (c - radius) * chunk)
                 hi = min(T, (c + radius + 1) * chunk)
-                F[b, h, c], G[b, h, c] = _scan_outside_window(stats, al, init, T, lo, hi)
+                F[b, h, c], G[b, h, c] = _scan_outside_window(stats, al, init, T, lo, hi,
+                                                              frozen)
     return F, G
 
 

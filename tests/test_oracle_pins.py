@@ -137,6 +137,81 @@ def test_frozen_state_rule_differs_at_second_order():
     assert 3.8 < r < 4.2
 
 
+def test_frozen_rule_is_the_sum_of_token_corrections_at_one_state():
+    """The frozen-state rule, written as the pages define it: every token's
+    correction beta_i k_i (v_i - S~^T k_i)^T is evaluated at the same decayed
+    state S~ and all are added (explicit loop over tokens, per-token gates)."""
+    rng = np.random.default_rng(11)
+    dk, dv, n = 6, 4, 9
+    K = rng.normal(size=(n, dk))
+    V = rng.normal(size=(n, dv))
+    S = rng.normal(size=(dk, dv))
+    beta = rng.uniform(0.1, 0.9, size=n)
+    alpha = rng.uniform(0.5, 1.0, size=dk)
+    St = alpha[:, None] * S
+    want = St.copy()
+    for i in range(n):
+        want += beta[i] * np.outer(K[i], V[i] - St.T @ K[i])
+    got = O.vda_update(S, K, V, beta, alpha, frozen=True)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_frozen_rule_one_token_is_the_classic_delta_rule():
+    """N = 1: S~ + beta k (v - S~^T k)^T, the one-token delta rule; VDA's
+    (I + beta k k^T)^-1 (S~ + beta k v^T) differs from it."""
+    rng = np.random.default_rng(12)
+    k = rng.normal(size=5)
+    v = rng.normal(size=3)
+    S = rng.normal(size=(5, 3))
+    want = S + 0.7 * np.outer(k, v - S.T @ k)
+    got = O.vda_update(S, k[None], v[None], 0.7, frozen=True)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    assert np.linalg.norm(O.vda_update(S, k[None], v[None], 0.7) - want) > 1e-3
+
+
+def test_frozen_transition_can_expand_where_vda_cannot():
+    """Proposition 1 holds for VDA only: with beta ||k||^2 = 3 the frozen
+    transition I - beta k k^T has an eigenvalue -2 (it amplifies the inherited
+    state), while (I + beta k k^T)^-1 has spectral norm <= 1."""
+    k = np.array([1.0, 0.0, 0.0])
+    S0 = np.zeros((3, 2))
+    dS = np.array([[1.0, 0.0], [0.0, 0.0], [0.0, 0.0]])
+    v = np.zeros(2)
+
+    def carried(frozen):
+        return (O.vda_update(S0 + dS, k[None], v[None], 3.0, frozen=frozen) -
+                O.vda_update(S0, k[None], v[None], 3.0, frozen=frozen))
+
+    assert np.isclose(np.linalg.norm(carried(True)), 2.0)
+    assert np.isclose(np.linalg.norm(carried(False)), 0.25)
+
+
+def test_frozen_and_vda_agree_for_small_writes_in_the_forward():
+    """Whole linear branch: the two rules agree to first order in beta and
+    differ at beta of order 1."""
+    import torch
+    from synth import CONFIGS, make_inputs
+    cfg = CONFIGS["tiny_f32"]
+    inp = make_inputs(cfg)
+    args = (inp["q"], inp["k"], inp["v"], None, inp["text_k"], inp["text_v"], cfg.T, cfg.N)
+    rows = np.arange(0, cfg.L, 7)
+
+    def run(beta, frozen):
+        a = list(args)
+        a[3] = torch.full((cfg.B, cfg.H, 1 + cfg.T), beta)
+        return O.linear_branch(*a, rows=rows, frozen=frozen)
+
+    def rel_gap(beta):
+        ref = run(beta, False)
+        return np.abs(run(beta, True) - ref).max() / np.abs(ref).max()
+
+    # the output is O(beta) and the gap O(beta^2): the relative gap halves
+    # with beta, and is large at beta of order 1
+    r = rel_gap(2e-4) / rel_gap(1e-4)
+    assert 1.9 < r < 2.1
+    assert rel_gap(0.9) > 1e-2
+
+
 # --- Regions, mask ------------------------------------------------------------
 
 def _brute_visible(tq, tk, T, C, r):
