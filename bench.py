@@ -187,6 +187,8 @@ def base_line(args, cfg, value, ms_per_step, n_gpus):
                    "text_keys_in_softmax": bool(getattr(args, "text_softmax", False)),
                    "write_gate": "per token" if getattr(args, "beta_per_token", False)
                                  else "per frame",
+                   "frame_rule": "frozen-state (comparison)"
+                                 if getattr(args, "frozen_state", False) else "VDA",
                    "linear_feature_map": "VDA-Prep in the step (3x3 spatial + 5-tap temporal "
                                          "conv, SiLU, L2; random filters)"
                                          if getattr(args, "prep", False) else "inputs prepared"},
@@ -240,9 +242,11 @@ def run_ours(args, cfg):
     inp = make_inputs(cfg, alpha_range=(0.9, 1.0) if args.alpha else None,
                       beta_per_token=args.beta_per_token)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    if args.frozen_state:  # keys scaled by 1/sqrt(N) (a reading of SANA-WM's frame-size scaling)
+        d["k"] = (d["k"].float() / float(cfg.N) ** 0.5).to(d["k"].dtype)
     p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], chunk=cfg.chunk,
                        window_radius=cfg.window_radius, text_softmax=args.text_softmax,
-                       beta_per_token=args.beta_per_token)
+                       beta_per_token=args.beta_per_token, frozen_state=args.frozen_state)
     ws = vdn.alloc_workspace(p)
     out = torch.empty(cfg.B, cfg.L, p.D_out, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -413,6 +417,8 @@ def main():
                     help="video queries also attend all text tokens in the Softmax branch")
     ap.add_argument("--beta-per-token", action="store_true",
                     help="one write gate per token instead of per frame")
+    ap.add_argument("--frozen-state", action="store_true",
+                    help="frame updates by the frozen-state comparison rule instead of VDA")
     ap.add_argument("--prep", action="store_true",
                     help="time VDA-Prep (linear-branch feature map of raw q, k, v) in every step")
     ap.add_argument("--alpha", action="store_true",

@@ -107,6 +107,13 @@ typedef struct CUstream_st *vdn_stream_t;
  * video tokens in token order.  On the tensor-core path the frame statistics
  * use sqrt(beta_i)-scaled fp16 copies of the key/value tiles. */
 #define VDN_FLAG_BETA_PER_TOKEN (1u << 3)
+/* Comparison mode: every frame update follows the frozen-state (SANA-WM)
+ * batched rule of the Video Delta Attention section instead of VDA's: all
+ * token corrections are evaluated at the same decayed state,
+ * S_t = (I - A_t) Diag(alpha_t) S_{t-1} + W_t (no inverse; the text frame
+ * likewise, S_text = W_text).  Keys are taken as given: SANA-WM's frame-size
+ * key scaling, whose factor the pages lost, is left to the caller. */
+#define VDN_FLAG_FROZEN_STATE (1u << 4)
 
 typedef struct vdn_params {
   int B;             /* batch */

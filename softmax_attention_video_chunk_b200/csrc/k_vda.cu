@@ -36,7 +36,7 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
                        const TIn* __restrict__ text_k, const TIn* __restrict__ text_v,
                        const float* __restrict__ beta, const float* __restrict__ alpha,
                        float* __restrict__ Mout, float* __restrict__ Rout, int H, int T,
-                       int N, int n_text, bool beta_tok) {
+                       int N, int n_text, bool beta_tok, bool frozen) {
   constexpr int RT = D / 16;  // rows per thread
   constexpr int CT = D / 16;  // cols per thread
   constexpr int BN = 16;      // tokens per staged tile
@@ -124,6 +124,19 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
     }
   }
   __syncthreads();
+  if (frozen) {  // frozen-state rule: M = (I - beta A) Diag(alpha), R = beta W
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const int i = ty * RT + r;
+#pragma unroll
+      for (int m = 0; m < CT; ++m) {
+        const int j = tx + 16 * m;
+        Mo[i * D + j] = ((i == j ? 1.f : 0.f) - bt * accA[r][m]) * (al ? al[j] : 1.f);
+        Ro[i * D + j] = bt * accW[r][m];
+      }
+    }
+    return;
+  }
   // [I + beta A | Diag(alpha) | beta W]
 #pragma unroll
   for (int r = 0; r < RT; ++r) {
@@ -425,7 +438,7 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<dim3(T + 1, H, B), 256, sm, st>>>(
         (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.text_k, (const TIn*)a.text_v, a.beta,
-        a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text, a.beta_tok);
+        a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text, a.beta_tok, a.frozen);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {

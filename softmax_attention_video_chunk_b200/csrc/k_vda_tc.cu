@@ -20,6 +20,8 @@
 //               pivot), then R = X W and M = X Diag(alpha) on CUDA cores (FP32).
 // For d = 64 the MMA computes [K|V]^T [K|V] (M = N = 128) and keeps the first
 // 64 rows.  Anchor frames write M = Diag(alpha), R = 0 and exit.
+// Frozen-state rule (comparison mode): X = I - beta A without the inversion,
+// M = X Diag(alpha) and R = beta W.
 // Per-token write gates: warps 2-7 turn every landed bf16 tile into an exact
 // fp16 copy (the A operand, in place) and into beta_i-scaled fp16 hi and lo
 // parts (two B operands: beta*x = hi + lo to ~22 bits); two MMA chains
@@ -42,6 +44,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_tv, const float* __restrict__ beta,
                     const float* __restrict__ alpha, float* __restrict__ Mout,
                     float* __restrict__ Rout, int H, int T, int N, int n_text, bool beta_tok,
+                    bool frozen,
                     int* __restrict__ status) {
   constexpr int BT = 64;                  // tokens per stage
   constexpr int NBLK = D / 32;            // 64-channel blocks of [K | V]
@@ -246,8 +249,8 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
         for (int e = 0; e < 32; ++e) {
           const int j = 32 * c + e;
           const float x = bt * __uint_as_float(r[e]);
-          if (part == 0)
-            Ash[i * SD + j] = x + (i == j ? 1.f : 0.f);
+          if (part == 0)  // I + beta A (VDA), or I - beta A (frozen-state rule)
+            Ash[i * SD + j] = (frozen ? -x : x) + (i == j ? 1.f : 0.f);
           else
             Wsh[i * SD + j] = x;
         }
@@ -269,7 +272,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
     for (int c = 0; c < BL; ++c) a[i][c] = Ash[(ty * BL + i) * SD + tx * BL + c];
   int buf = 0;
-  for (int pb = 0; pb < 16; ++pb) {
+  for (int pb = 0; pb < (frozen ? 0 : 16); ++pb) {  // the frozen-state rule has no inverse
 #pragma unroll
     for (int r = 0; r < BL; ++r) {
       const int p = pb * BL + r;
@@ -317,6 +320,17 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
       m4.w = a[i][c + 3] * (al ? al[tx * BL + c + 3] : 1.f);
       *reinterpret_cast<float4*>(dst + c) = m4;
     }
+  }
+  if (frozen) {  // R = beta W (uniform over the CTA)
+#pragma unroll
+    for (int i = 0; i < BL; ++i) {
+      float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
+      const float* src = Wsh + (ty * BL + i) * SD + tx * BL;
+#pragma unroll
+      for (int c = 0; c < BL; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(src[c], src[c + 1], src[c + 2], src[c + 3]);
+    }
+    return;
   }
   __syncthreads();
 #pragma unroll
@@ -383,7 +397,8 @@ static cudaError_t launch_frame_tc_t(const VdaArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.T + 1, a.H, a.B), 256, sm, st>>>(mk, mv, mtk, mtv, a.beta, a.alpha, a.Mf, a.Rf,
-                                                 a.H, a.T, a.N, a.n_text, a.beta_tok, a.status);
+                                                 a.H, a.T, a.N, a.n_text, a.beta_tok, a.frozen,
+                                                 a.status);
   return cudaGetLastError();
 }
 

@@ -65,7 +65,7 @@ static WsLayout layout(const vdn_params& p) {
 static vdn_status validate_params(const vdn_params* p) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;
   if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT | VDN_FLAG_TEXT_SOFTMAX |
-                             VDN_FLAG_BETA_PER_TOKEN))
+                             VDN_FLAG_BETA_PER_TOKEN | VDN_FLAG_FROZEN_STATE))
     return VDN_ERR_INVALID_ARG;
   if ((p->dtype != VDN_F32 && p->dtype != VDN_BF16) ||
       (p->out_dtype != VDN_F32 && p->out_dtype != VDN_BF16))
@@ -146,6 +146,7 @@ static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const
   a.FS = (float*)(ws + w.FS); a.GS = (float*)(ws + w.GS);
   a.tc = use_tc(*p);
   a.beta_tok = (p->flags & VDN_FLAG_BETA_PER_TOKEN) != 0;
+  a.frozen = (p->flags & VDN_FLAG_FROZEN_STATE) != 0;
   a.status = (int*)(ws + w.status);
   return a;
 }

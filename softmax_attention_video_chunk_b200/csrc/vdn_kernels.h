@@ -18,6 +18,7 @@ struct VdaArgs {
   float *Mf, *Rf, *CM, *CR, *FS, *GS;
   bool tc;      // frame statistics on the tensor cores (bf16, d in {64, 128})
   bool beta_tok;  // beta per token: [B][H][n_text + L]
+  bool frozen;    // frozen-state rule: M = (I - A) Diag(alpha), R = W (no inverse)
   int* status;  // device status word
 };
 

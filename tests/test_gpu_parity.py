@@ -137,6 +137,54 @@ def test_edge_cases(name, over, mk, kw, simt):
     assert e_l <= 1e-4
 
 
+def _frozen_inputs(cfg):
+    """Inputs for the frozen-state comparison rule: keys scaled by 1/sqrt(N),
+    one reading of SANA-WM's frame-size key scaling, so that the frame
+    transitions I - A stay near the unit ball over the clip."""
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0))
+    inp["k"] = (inp["k"].float() / np.sqrt(cfg.N)).to(inp["k"].dtype)
+    return inp
+
+
+@pytest.mark.parametrize("simt", [False, True])
+@pytest.mark.parametrize("over", [dict(T=14, N=72), dict(T=9, N=130, d=128, H=2, n_text=37)],
+                         ids=["d64", "d128"])
+def test_frozen_state_rule(over, simt):
+    """Comparison mode: every frame update follows the frozen-state rule."""
+    cfg = _edge_cfg(over)
+    inp = _frozen_inputs(cfg)
+    d = to_dev(inp)
+    out = _fwd(d, cfg, simt=simt, frozen_state=True)
+    _, o_l = _branches(d, cfg, simt=simt, frozen_state=True, want_soft=False)
+    torch.cuda.synchronize()
+    want, _, wl_ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius, frozen=True)
+    e_out, e_l = rel_err(out.double().cpu(), want), rel_err(o_l.double().cpu(), wl_)
+    # and it is a different rule: VDA's o_lin differs from it
+    _, vda_l = _branches(d, cfg, simt=simt, want_soft=False)
+    torch.cuda.synchronize()
+    gap = rel_err(vda_l.double().cpu(), wl_)
+    print(f"frozen {over} simt={simt}: out {e_out:.2e} o_lin {e_l:.2e} (VDA gap {gap:.2e})")
+    assert e_out <= TOL_OUT["bf16"]
+    assert e_l <= 1e-4
+    assert gap > 1e-2
+
+
+@pytest.mark.parametrize("over", [dict(T=23, N=96, d=64, H=2), dict(T=12, N=136, d=128, H=2)],
+                         ids=["d64", "d128"])
+def test_boundary_states_frozen(over):
+    cfg = _edge_cfg(over)
+    inp = _frozen_inputs(cfg)
+    d = to_dev(inp)
+    F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
+                                   alpha=d["alpha"], chunk=cfg.chunk, frozen_state=True)
+    torch.cuda.synchronize()
+    Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+                               cfg.T, cfg.N, cfg.chunk, alpha=inp["alpha"], frozen=True)
+    eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
+    print(f"frozen states {over}: F {eF:.2e} G {eG:.2e}")
+    assert eF <= 1e-4 and eG <= 1e-4
+
+
 def test_wide_scores_rescale_path():
     """Scores spanning many octaves (q scaled up): the running-max rescale of
     the tensor-core kernel is exercised."""
