@@ -219,6 +219,23 @@ def run_reference(args, cfg):
     return 0
 
 
+def ranks_max(x: float, dist, device) -> float:
+    """Max of x over all ranks (x itself when no process group is up): every
+    multi-GPU time is the slowest rank's."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, elapsed_ms: float) -> float:
+    """Units per second over all ranks: each of the `world` replicas processed
+    `units_per_rank_step` units in each of `steps` steps within elapsed_ms."""
+    return world * units_per_rank_step * steps / (elapsed_ms / 1e3)
+
+
 def run_ours(args, cfg):
     import torch
     import softmax_attention_video_chunk_b200 as vdn
@@ -299,10 +316,7 @@ def run_ours(args, cfg):
     elapsed_ms = t_start.elapsed_time(t_end)
     stage_ms = [sum(evs[i][s].elapsed_time(evs[i][s + 1]) for i in range(args.steps)) / args.steps
                 for s in range(nS)]
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = ranks_max(elapsed_ms, dist, "cuda")
     st = vdn.device_status(p, ws)
     if st != 0:
         raise RuntimeError(f"device status after timing: {vdn.STATUS[st]}")
@@ -316,7 +330,7 @@ def run_ours(args, cfg):
 
     ms_per_step = elapsed_ms / args.steps
     tokens = cfg.B * cfg.L
-    value = world * tokens * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, tokens, args.steps, elapsed_ms)
 
     # ---- end to end: pinned host inputs -> device, forward, result -> host,
     # through the pipelined host API (uploads, compute and download of
@@ -342,11 +356,8 @@ def run_ours(args, cfg):
     e1.record(pipe.s_d2h)
     pipe.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * tokens * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = ranks_max(e2e_ms, dist, "cuda")
+    e2e_value = whole_job_rate(world, tokens, e2e_steps, e2e_ms)
 
     if rank == 0:
         wm = work_model(cfg, text_keys=args.text_softmax)
