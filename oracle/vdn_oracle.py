@@ -163,6 +163,30 @@ def softmax_branch(q, k, v, T, N, chunk=5, radius=1, scale=None, rows=None,
     return out
 
 
+def text_query_branch(text_q, k, v, text_k, text_v, scale=None, rows=None):
+    """Softmax attention of the text tokens as queries: every text query sees
+    every video key and every text key under one normaliser, with no mask
+    (reading of the joint Softmax with text: text rows are dense over the
+    clip).  text_q, text_k, text_v [B, n_text, H, d]; k, v [B, L, H, d].
+    Returns [B, R, H, d_v] for the selected text rows."""
+    tq = np.asarray(text_q, F64)
+    kk = np.concatenate([np.asarray(k, F64), np.asarray(text_k, F64)], axis=1)
+    vv = np.concatenate([np.asarray(v, F64), np.asarray(text_v, F64)], axis=1)
+    B, nt, H, dk = tq.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    rows = np.arange(nt) if rows is None else np.asarray(rows)
+    out = np.zeros((B, len(rows), H, vv.shape[-1]), F64)
+    for b in range(B):
+        for h in range(H):
+            s = scale * (tq[b, rows, h, :] @ kk[b, :, h, :].T)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, :, h, :] = p @ vv[b, :, h, :]
+    return out
+
+
 # ----------------------------------------------------------------------------
 # Video Delta Attention
 # ----------------------------------------------------------------------------

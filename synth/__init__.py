@@ -5,4 +5,4 @@ CUDA path and the CPU oracle consume.  It contains none of the method's
 arithmetic.
 """
 from .inputs import (CONFIGS, Config, grid_shape, make_inputs, make_prep_inputs,  # noqa: F401
-                     sample_rows)
+                     make_text_queries, sample_rows)

@@ -203,3 +203,15 @@ def make_prep_inputs(cfg: Config, *, grid: Optional[tuple] = None, device: str =
     if device != "cpu":
         out = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in out.items()}
     return out
+
+
+def make_text_queries(cfg: Config, *, device: str = "cpu") -> torch.Tensor:
+    """Text-token queries [B, n_text, H, d] for the text rows of the joint
+    Softmax, from a third seeded generator (seed + 104729, so no other draw
+    changes): N(0, 1), L2-normalised per (token, head) when ``q_norm`` is set,
+    rounded once to the workload dtype."""
+    g = torch.Generator(device="cpu").manual_seed(cfg.seed + 104729)
+    tq = torch.randn(cfg.B, cfg.n_text, cfg.H, cfg.d, generator=g, dtype=torch.float32)
+    if cfg.q_norm:
+        tq = _l2n(tq)
+    return tq.to(_TORCH_DTYPE[cfg.dtype]).to(device)

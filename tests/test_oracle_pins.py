@@ -212,6 +212,32 @@ def test_frozen_and_vda_agree_for_small_writes_in_the_forward():
     assert rel_gap(0.9) > 1e-2
 
 
+def test_text_queries_dense_softmax_matches_library_attention():
+    """Text rows: dense attention over [video keys; text keys], against
+    torch's scaled_dot_product_attention on the concatenated keys."""
+    import torch
+    rng = np.random.default_rng(21)
+    B, L, nt, H, d = 2, 37, 9, 3, 8
+    tq, k, v = (rng.normal(size=(B, n, H, d)) for n in (nt, L, L))
+    tk, tv = (rng.normal(size=(B, nt, H, d)) for _ in range(2))
+    got = O.text_query_branch(tq, k, v, tk, tv)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(np.swapaxes(x, 1, 2)))  # [B, H, n, d]
+    want = torch.nn.functional.scaled_dot_product_attention(
+        t(tq), torch.cat([t(k), t(tk)], 2), torch.cat([t(v), t(tv)], 2))
+    np.testing.assert_allclose(got, np.swapaxes(want.numpy(), 1, 2), rtol=1e-10, atol=1e-12)
+
+
+def test_text_queries_single_key_returns_its_value():
+    rng = np.random.default_rng(22)
+    tq = rng.normal(size=(1, 4, 1, 5))
+    k, v = rng.normal(size=(1, 1, 1, 5)), rng.normal(size=(1, 1, 1, 5))
+    empty = np.zeros((1, 0, 1, 5))
+    # no text keys: the only key's value, for every text query
+    kk = np.concatenate([k, empty], 1)
+    out = O.text_query_branch(tq, kk, v, empty, empty)
+    np.testing.assert_allclose(out, np.broadcast_to(v, out.shape), rtol=1e-14)
+
+
 # --- Regions, mask ------------------------------------------------------------
 
 def _brute_visible(tq, tk, T, C, r):
