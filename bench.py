@@ -277,6 +277,11 @@ def run_ours(args, cfg):
                                   cfg.dtype)
         prep_ws = torch.zeros(vdn.PREP_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
     prep_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    tq = None
+    if args.text_softmax:  # text queries too: the text rows of the joint Softmax
+        from synth import make_text_queries
+        tq = make_text_queries(cfg).cuda()
+    tq_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
 
     def step(events=None, i=None):
         if lin is not None:
@@ -290,6 +295,13 @@ def run_ours(args, cfg):
         vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
                             d["W_soft"], d["W_lin"], d["gates"], cfg.T, alpha=d["alpha"],
                             out=out, workspace=ws, params=p, events=events, lin=lin)
+        if tq is not None:  # the text rows of the joint Softmax (dense over every key)
+            if i is not None:
+                tq_ev[i][0].record(stream)
+            vdn.text_query_attn(tq, d["k"], d["v"], d["text_k"], d["text_v"], cfg.T,
+                                workspace=ws, params=p)
+            if i is not None:
+                tq_ev[i][1].record(stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -320,6 +332,9 @@ def run_ours(args, cfg):
     st = vdn.device_status(p, ws)
     if st != 0:
         raise RuntimeError(f"device status after timing: {vdn.STATUS[st]}")
+    tq_ms = None
+    if tq is not None:
+        tq_ms = sum(e[0].elapsed_time(e[1]) for e in tq_ev) / args.steps
     prep_ms = None
     if lin is not None:
         prep_ms = sum(e[0].elapsed_time(e[1]) for e in prep_ev) / args.steps
@@ -385,6 +400,9 @@ def run_ours(args, cfg):
         line["stages_ms"] = dict(zip(vdn.STAGE_NAMES, [round(x, 4) for x in stage_ms]))
         line["gpu_launches"] = args.steps * ((8 if vdn.use_tc_params(p) else 6) +
                                              (2 if prep_ms is not None else 0))
+        if tq_ms is not None:
+            line["stages_ms"]["text_rows"] = round(tq_ms, 4)
+            line["gpu_launches"] += args.steps * 2  # V^T conversion + text-row Softmax
         if prep_ms is not None:
             es = 2 if cfg.dtype == "bf16" else 4
             prep_bytes = 6 * cfg.B * cfg.L * cfg.H * cfg.d * es  # read q, k, v; write 3

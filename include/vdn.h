@@ -249,6 +249,24 @@ VDN_API vdn_status vdn_vda_prep(const vdn_prep_params *p, const void *q, const v
                                 void *v_out, void *workspace, size_t workspace_bytes,
                                 vdn_stream_t stream);
 
+/* Text tokens as queries: the text rows of the joint Softmax with text
+ * (method section: the text keeps its Softmax path).  Every text query
+ * attends every video key and every text key under one normaliser, with no
+ * mask:  o_text[i] = softmax_j(scale * q_i . k_j) v_j  over j in
+ * [video tokens; text tokens].
+ *  - text_q: [B, n_text, H, d] dtype params.dtype (the text tokens' queries);
+ *    k, v: [B, L, H, d]; text_k, text_v: [B, n_text, H, d].
+ *  - o_text: float32 [B, n_text, H, d_v], caller-owned.
+ *  - Needs n_text >= 1 (else VDN_ERR_SHAPE).  The workspace must hold
+ *    vdn_workspace_bytes of the same params with VDN_FLAG_TEXT_SOFTMAX set
+ *    (the transposed text values live there).  Runs the tensor-core kernel
+ *    for bf16 with d in {64, 128}, the FP32 kernel otherwise (or with
+ *    VDN_FLAG_SIMT).  Other conventions as vdn_hybrid_attn_fwd. */
+VDN_API vdn_status vdn_text_query_attn(const vdn_params *p, const void *text_q, const void *k,
+                                       const void *v, const void *text_k, const void *text_v,
+                                       float *o_text, void *workspace, size_t workspace_bytes,
+                                       vdn_stream_t stream);
+
 /* The two branch readouts before gating and projection, float32
  * [B, L, H, d_v]: o_soft = Softmax branch, o_lin = linear branch before its
  * RMS norm.  Either output pointer may be NULL to skip that branch. */

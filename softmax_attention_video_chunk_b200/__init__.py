@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_prep_params_init.argtypes = [PPP] + [ctypes.c_int] * 7
         L.vdn_vda_prep.restype = ctypes.c_int
         L.vdn_vda_prep.argtypes = [PPP] + [_P] * 11 + [ctypes.c_size_t, _P]
+        L.vdn_text_query_attn.restype = ctypes.c_int
+        L.vdn_text_query_attn.argtypes = [PP] + [_P] * 7 + [ctypes.c_size_t, _P]
         L.vdn_selftest_bounded_wait.restype = ctypes.c_int
         L.vdn_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint, _P]
         _lib = L
@@ -223,6 +225,22 @@ def hybrid_attn_fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, *, a
     if rc != 0:
         raise VdnError(rc, "vdn_hybrid_attn_fwd")
     return out
+
+
+def text_query_attn(text_q, k, v, text_k, text_v, T, *, workspace=None, stream=None,
+                    params=None, **kw):
+    """o_text float32 [B, n_text, H, d]: the text tokens as queries over every
+    video and text key (vdn_text_query_attn)."""
+    import torch
+    kw["text_softmax"] = True  # workspace with the text tokens' V^T
+    p = params or params_for(k, v, text_k, T, **kw)
+    o = torch.empty(text_q.shape, dtype=torch.float32, device=text_q.device)
+    ws = alloc_workspace(p, k.device) if workspace is None else workspace
+    rc = lib().vdn_text_query_attn(ctypes.byref(p), _ptr(text_q), _ptr(k), _ptr(v), _ptr(text_k),
+                                   _ptr(text_v), _ptr(o), _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_text_query_attn")
+    return o
 
 
 def make_prep_params(B, H, T, grid_h, grid_w, d, dtype="bf16", l2_eps=1e-6) -> VdnPrepParams:

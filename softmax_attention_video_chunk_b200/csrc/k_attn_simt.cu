@@ -23,16 +23,27 @@ __global__ void __launch_bounds__(128)
 attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                  const TIn* __restrict__ v, const TIn* __restrict__ tk,
                  const TIn* __restrict__ tv, int n_text, float* __restrict__ o, Geo geo,
-                 int H, float scale) {
+                 int H, float scale, const TIn* __restrict__ qt) {
   constexpr int BQ = 32, BK = 32, QS = D + 4;
   constexpr int NO = D / 16;  // float4 output groups per thread
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int L = geo.T * geo.N;
   QGroup g;
   int row_start;
-  if (!find_tile(geo, BQ, blockIdx.x, &g, &row_start)) return;
-  const int L = geo.T * geo.N;
+  if (qt != nullptr) {  // text queries: one dense group over every video key
+    g.row0 = 0; g.nrows = n_text; g.nseg = 1;
+    g.seg0[0] = 0; g.seg1[0] = L;
+    g.seg0[1] = g.seg1[1] = g.seg0[2] = g.seg1[2] = 0;
+    row_start = blockIdx.x * BQ;
+    if (row_start >= n_text) return;
+  } else if (!find_tile(geo, BQ, blockIdx.x, &g, &row_start)) {
+    return;
+  }
   const size_t rs = (size_t)H * D;
-  const size_t base = (size_t)b * L * rs + (size_t)h * D;
+  const size_t base = (size_t)b * L * rs + (size_t)h * D;           // video tokens
+  const size_t tbase = (size_t)b * n_text * rs + (size_t)h * D;     // text tokens
+  const TIn* qsrc = qt != nullptr ? qt : q;
+  const size_t qbase = qt != nullptr ? tbase : base;                 // query rows / output
 
   extern __shared__ __align__(16) float sm_attn[];
   float* Qs = sm_attn;         // [BQ][QS]
@@ -44,7 +55,7 @@ attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   for (int e = tid; e < BQ * D; e += blockDim.x) {
     const int r = e / D, c = e % D;
     const int row = min(row_start + r, row_end - 1);
-    Qs[r * QS + c] = to_f(q[base + (size_t)row * rs + c]) * scale;
+    Qs[r * QS + c] = to_f(qsrc[qbase + (size_t)row * rs + c]) * scale;
   }
 
   const int r = tid >> 2, sub = tid & 3;
@@ -54,7 +65,6 @@ attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   for (int gq = 0; gq < NO; ++gq) acc[gq][0] = acc[gq][1] = acc[gq][2] = acc[gq][3] = 0.f;
 
   // key ranges of the group, then (optionally) the text tokens as one more range
-  const size_t tbase = (size_t)b * n_text * rs + (size_t)h * D;
   for (int s = 0; s < g.nseg + (n_text > 0 ? 1 : 0); ++s) {
     const bool text = s == g.nseg;
     const TIn* ks = text ? tk : k;
@@ -127,7 +137,7 @@ attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   }
   if (row_start + r < row_end) {
     const float inv = 1.f / l_run;
-    float* dst = o + base + (size_t)(row_start + r) * rs;
+    float* dst = o + qbase + (size_t)(row_start + r) * rs;
 #pragma unroll
     for (int gq = 0; gq < NO; ++gq)
       *reinterpret_cast<float4*>(dst + sub * 4 + 16 * gq) =
@@ -138,14 +148,14 @@ attn_simt_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 template <int D, typename TIn>
 static cudaError_t launch_t(const AttnArgs& a, float* o, cudaStream_t st) {
   Geo geo{a.T, a.N, a.C, a.R};
-  const int tiles = count_tiles(geo, 32);
+  const int tiles = a.text_q != nullptr ? (a.n_text_keys + 31) / 32 : count_tiles(geo, 32);
   const size_t sm = sizeof(float) * (2 * 32 * (D + 4) + 32 * D + 32 * 33);
   auto kern = attn_simt_kernel<D, TIn>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   kern<<<dim3(tiles, a.H, a.B), 128, sm, st>>>(
       (const TIn*)a.q, (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.text_k,
-      (const TIn*)a.text_v, a.n_text_keys, o, geo, a.H, a.scale);
+      (const TIn*)a.text_v, a.n_text_keys, o, geo, a.H, a.scale, (const TIn*)a.text_q);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,8 @@
 //               by more than 2^8) and row sum, writes P = 2^(s - m) as fp16
 //               over its S columns, and finally normalises O and writes
 //               g_s * o_s (fp16, the projection operand) or o_s (fp32).
+// Text queries (n_qtext > 0): the same kernel runs the text tokens' rows as
+// one dense group over every video key plus the text keys (o_s output only).
 // TMEM (512 columns): S0 | S1 | O0 | O1.  Every mbarrier wait is bounded in
 // time; on expiry the CTA records VDN_ERR_TIMEOUT in the status word, drains
 // its MMAs and copies, frees TMEM and exits.
@@ -125,7 +127,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                const __grid_constant__ CUtensorMap map_tk,
                const __grid_constant__ CUtensorMap map_tvt, int n_text, Geo geo, int B, int H,
                float scale_log2, const __nv_bfloat16* __restrict__ gates,
-               __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status) {
+               __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status,
+               int n_qtext) {
   constexpr int BM = 128, NS = 2;
   constexpr int QT = BM * D * 2;   // bytes of a Q tile
   constexpr int KT = kBK * D * 2;  // bytes of a K tile
@@ -155,7 +158,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
   const int b = bh / H, h = bh % H;
   QGroup g;
   int row0;
-  if (!find_tile(geo, 2 * BM, pair, &g, &row0)) return;  // uniform over the CTA
+  if (n_qtext > 0) {  // text queries: one dense group over every video key
+    g.row0 = 0; g.nrows = n_qtext; g.nseg = 1;
+    g.seg0[0] = 0; g.seg1[0] = geo.T * geo.N;
+    g.seg0[1] = g.seg1[1] = g.seg0[2] = g.seg1[2] = 0;
+    row0 = pair * 2 * BM;
+    if (row0 >= n_qtext) return;  // uniform over the CTA
+  } else if (!find_tile(geo, 2 * BM, pair, &g, &row0)) {
+    return;  // uniform over the CTA
+  }
   const int row_end = g.row0 + g.nrows;
   const bool has1 = row0 + BM < row_end;
   const int n_video = kv_count(g);
@@ -434,7 +445,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int row = row0 + j * BM + wq * 32 + lane;
         const bool valid = row < row_end;
         const float inv = 1.f / l_sum;
-        const size_t tok = (size_t)b * L + row;
+        const size_t tok = (size_t)b * (n_qtext > 0 ? n_qtext : L) + row;
         bool bad = false;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -494,9 +505,19 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
     const uint64_t dims[4] = {(uint64_t)D, H, L, B};
     const uint64_t str[3] = {(uint64_t)D * 2, H * D * 2, L * H * D * 2};
     const uint32_t box[4] = {64, 1, 128, 1};
-    if (!make_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.q, dims, str, box))
-      return cudaErrorInvalidValue;
     if (!make_tmap(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.k, dims, str, box))
+      return cudaErrorInvalidValue;
+    if (t.text_q == nullptr &&
+        !make_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.q, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  const int n_qtext = t.text_q != nullptr ? t.n_text_keys : 0;
+  if (n_qtext > 0) {  // queries are the text tokens [B, n_text, H, D]
+    const uint64_t nt = (uint64_t)n_qtext;
+    const uint64_t dims[4] = {(uint64_t)D, H, nt, B};
+    const uint64_t str[3] = {(uint64_t)D * 2, H * D * 2, nt * H * D * 2};
+    const uint32_t box[4] = {64, 1, 128, 1};
+    if (!make_tmap(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.text_q, dims, str, box))
       return cudaErrorInvalidValue;
   }
   {
@@ -521,7 +542,7 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
       return cudaErrorInvalidValue;
   }
   Geo geo{t.T, t.N, t.C, t.R};
-  const int pairs = count_tiles(geo, 256);
+  const int pairs = n_qtext > 0 ? (n_qtext + 255) / 256 : count_tiles(geo, 256);
   const size_t sm = 1024 + 2 * (128 * D * 2) + 2 * 2 * (128 * D * 2) + 256;
   auto kern = attn_tc_kernel<D, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -530,11 +551,12 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
   const unsigned grid = (unsigned)pairs * (unsigned)(t.B * t.H);
   kern<<<grid, 320, sm, st>>>(mq, mk, mv, mtk, mtv, t.n_text_keys, geo, t.B, t.H, scale_log2,
                               FUSED ? (const __nv_bfloat16*)f->gates : nullptr,
-                              FUSED ? f->x : nullptr, o_s, t.status);
+                              FUSED ? f->x : nullptr, o_s, t.status, n_qtext);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const TcAttnArgs& t, const TcFwdArgs* f, float* o_s, cudaStream_t st) {
+  if (f != nullptr && t.text_q != nullptr) return cudaErrorInvalidValue;  // text rows: o_s only
   if (f != nullptr) {
     if (t.D == 128) return launch_attn_t<128, true>(t, f, nullptr, st);
     if (t.D == 64) return launch_attn_t<64, true>(t, f, nullptr, st);

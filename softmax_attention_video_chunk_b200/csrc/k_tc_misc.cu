@@ -102,7 +102,7 @@ TcAttnArgs tc_attn_args(const vdn_params& p, const AttnArgs& a, void* vt, int* s
   t.scale = a.scale; t.q = a.q; t.k = a.k; t.v = a.v; t.vt = (__half*)vt; t.status = status;
   t.n_text_keys = a.n_text_keys;
   t.ntp = (int)round_up((size_t)a.n_text_keys, 64);
-  t.text_k = a.text_k; t.text_v = a.text_v;
+  t.text_k = a.text_k; t.text_v = a.text_v; t.text_q = a.text_q;
   t.vt_text = t.vt + (size_t)t.B * t.H * t.D * t.Lp;
   return t;
 }

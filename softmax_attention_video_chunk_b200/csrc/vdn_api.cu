@@ -456,6 +456,33 @@ vdn_status vdn_vda_prep(const vdn_prep_params* p, const void* q, const void* k, 
   return VDN_OK;
 }
 
+vdn_status vdn_text_query_attn(const vdn_params* p, const void* text_q, const void* k,
+                               const void* v, const void* text_k, const void* text_v,
+                               float* o_text, void* workspace, size_t workspace_bytes,
+                               vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  if (p->n_text < 1) return VDN_ERR_SHAPE;
+  const void* need[6] = {text_q, k, v, text_k, text_v, o_text};
+  for (const void* ptr : need) VDN_TRY(check_ptr(ptr, true));
+  vdn_params pt = *p;  // the text tokens join the keys (their V^T in the workspace)
+  pt.flags |= VDN_FLAG_TEXT_SOFTMAX;
+  VDN_TRY(check_ws(&pt, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  const WsLayout w = layout(pt);
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  AttnArgs a = attn_args(&pt, nullptr, k, v, text_k, text_v);
+  a.text_q = text_q;
+  if (use_tc(pt)) {
+    TcAttnArgs t = tc_attn_args(pt, a, ws + w.vt, (int*)(ws + w.status));
+    VDN_CUDA(launch_convert_v(t, st));
+    VDN_CUDA(launch_attn_tc(t, nullptr, o_text, st));
+  } else {
+    VDN_CUDA(launch_attn_simt(a, o_text, st));
+  }
+  return VDN_OK;
+}
+
 vdn_status vdn_device_status(const vdn_params* p, void* workspace, vdn_stream_t stream) {
   if (p != nullptr) VDN_TRY(validate_params(p));
   if (workspace == nullptr) return VDN_ERR_WORKSPACE;

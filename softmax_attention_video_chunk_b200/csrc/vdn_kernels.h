@@ -35,6 +35,7 @@ struct AttnArgs {
   const void *q, *k, *v;
   int n_text_keys;                  // text tokens joining the Softmax keys (0: none)
   const void *text_k, *text_v;      // [B, n_text, H, D]
+  const void* text_q = nullptr;     // text queries [B, n_text, H, D]: dense text rows
 };
 cudaError_t launch_attn_simt(const AttnArgs& a, float* o_s, cudaStream_t st);
 

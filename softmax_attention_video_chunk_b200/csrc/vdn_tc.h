@@ -23,6 +23,7 @@ struct TcAttnArgs {
   int ntp;                // n_text_keys rounded up to 64
   const void *text_k, *text_v;  // bf16 [B, n_text, H, D]
   __half* vt_text;        // fp16 [B*H][D][ntp], text V transposed
+  const void* text_q = nullptr;  // bf16 [B, n_text, H, D]: text queries (dense rows)
 };
 
 struct TcFwdArgs {

@@ -11,7 +11,7 @@ import torch
 
 import softmax_attention_video_chunk_b200 as vdn
 from oracle import vdn_oracle as O
-from synth import CONFIGS, make_inputs, sample_rows
+from synth import CONFIGS, make_inputs, make_text_queries, sample_rows
 from tests._parity import TOL_OUT, gpu_rows, oracle_forward, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -183,6 +183,45 @@ def test_boundary_states_frozen(over):
     eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
     print(f"frozen states {over}: F {eF:.2e} G {eG:.2e}")
     assert eF <= 1e-4 and eG <= 1e-4
+
+
+@pytest.mark.parametrize("simt", [False, True])
+@pytest.mark.parametrize("over", [dict(T=13, N=72, n_text=200), dict(T=9, N=130, d=128, H=2,
+                                  n_text=300), dict(T=5, N=16, n_text=3)],
+                         ids=["d64_nt200", "d128_nt300", "nt3"])
+def test_text_query_rows(over, simt):
+    """Text tokens as queries, dense over every video key and text key."""
+    cfg = _edge_cfg(over)
+    inp = make_inputs(cfg)
+    tq = make_text_queries(cfg)
+    d = to_dev(inp)
+    o = vdn.text_query_attn(tq.cuda(), d["k"], d["v"], d["text_k"], d["text_v"], cfg.T, simt=simt)
+    torch.cuda.synchronize()
+    want = O.text_query_branch(O._to_np(tq), O._to_np(inp["k"]), O._to_np(inp["v"]),
+                               O._to_np(inp["text_k"]), O._to_np(inp["text_v"]))
+    e = rel_err(o.double().cpu(), want)
+    print(f"text rows {over} simt={simt}: {e:.2e}")
+    # tensor cores: P rounded once to fp16 (as for the video rows); FP32 kernel: exact
+    assert e <= (1e-5 if simt else 2e-3)
+
+
+def test_text_query_rows_768p_sampled():
+    """768p: 512 text queries over 115200 video keys + 512 text keys; sampled rows."""
+    cfg = CONFIGS["768p_bf16"]
+    inp = make_inputs(cfg)
+    tq = make_text_queries(cfg)
+    d = to_dev(inp)
+    o = vdn.text_query_attn(tq.cuda(), d["k"], d["v"], d["text_k"], d["text_v"], cfg.T)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 137, 255, 256, 400, 510, 511])
+    got = o[:, rows].double().cpu().numpy()
+    del d, o
+    torch.cuda.empty_cache()
+    want = O.text_query_branch(O._to_np(tq), O._to_np(inp["k"]), O._to_np(inp["v"]),
+                               O._to_np(inp["text_k"]), O._to_np(inp["text_v"]), rows=rows)
+    e = rel_err(got, want)
+    print(f"768p text rows ({len(rows)} rows): {e:.2e}")
+    assert e <= 2e-3
 
 
 def test_wide_scores_rescale_path():
