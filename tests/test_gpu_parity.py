@@ -224,6 +224,20 @@ def test_text_query_rows_768p_sampled():
     assert e <= 2e-3
 
 
+def test_ulysses_one_rank_runs_the_library_forward():
+    """The head-sharded wrapper with its default per-rank forward (the CUDA
+    library) on one rank is the plain forward."""
+    from softmax_attention_video_chunk_b200 import ulysses
+    cfg = _edge_cfg(dict(T=10, N=48))
+    d = to_dev(make_inputs(cfg))
+    args = (d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], d["W_soft"],
+            d["W_lin"], d["gates"], cfg.T)
+    a = ulysses.ulysses_forward(*args)
+    b = vdn.hybrid_attn_fwd(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 def test_wide_scores_rescale_path():
     """Scores spanning many octaves (q scaled up): the running-max rescale of
     the tensor-core kernel is exercised."""

@@ -1,0 +1,100 @@
+"""Head-sharded (Ulysses) forward on CPU ranks with the gloo backend: the
+all-to-all / partial projection / reduce-scatter plumbing, with the float64
+oracle as each rank's forward, must reproduce the unsharded forward."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _cfg():
+    from synth import CONFIGS
+    return CONFIGS["tiny_f32"].replace(H=4)
+
+
+def _oracle_fwd(cfg):
+    from oracle import vdn_oracle as O
+
+    def fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, alpha=None, **kw):
+        inp = dict(q=q, k=k, v=v, beta=beta, alpha=alpha, text_k=text_k, text_v=text_v,
+                   W_soft=W_soft, W_lin=W_lin, gates=gates)
+        out, _, _ = O.hybrid_forward(inp, T, cfg.N, cfg.chunk, cfg.window_radius, **kw)
+        return torch.from_numpy(out)
+    return fwd
+
+
+def _rank(rank, world, port, out, alpha):
+    import datetime
+
+    import torch.distributed as dist
+
+    from softmax_attention_video_chunk_b200 import ulysses
+    from synth import make_inputs
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        cfg = _cfg()
+        inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None)
+        Ls = cfg.L // world
+        tok = slice(rank * Ls, (rank + 1) * Ls)
+        y = ulysses.ulysses_forward(
+            inp["q"][:, tok], inp["k"][:, tok], inp["v"][:, tok], inp["beta"], inp["text_k"],
+            inp["text_v"], inp["W_soft"], inp["W_lin"], inp["gates"][:, :, tok], cfg.T,
+            alpha=inp["alpha"], fwd=_oracle_fwd(cfg))
+        parts = [torch.empty_like(y) for _ in range(world)]
+        dist.all_gather(parts, y)
+        if rank == 0:
+            out["y"] = torch.cat(parts, dim=1).numpy()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,alpha", [(2, False), (4, True)])
+def test_head_sharded_forward_equals_unsharded(world, alpha):
+    from synth import make_inputs
+    cfg = _cfg()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(world, _free_port(), out, alpha), nprocs=world, join=True)
+        got = out["y"]
+    inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None)
+    want = _oracle_fwd(cfg)(inp["q"], inp["k"], inp["v"], inp["beta"], inp["text_k"],
+                            inp["text_v"], inp["W_soft"], inp["W_lin"], inp["gates"], cfg.T,
+                            alpha=inp["alpha"]).numpy()
+    rms = np.sqrt(np.mean(want ** 2))
+    assert got.shape == want.shape
+    assert np.max(np.abs(got - want)) <= 1e-12 * rms
+
+
+def test_one_rank_is_the_plain_forward():
+    from softmax_attention_video_chunk_b200 import ulysses
+    from synth import make_inputs
+    cfg = _cfg()
+    inp = make_inputs(cfg)
+    fwd = _oracle_fwd(cfg)
+    args = (inp["q"], inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+            inp["W_soft"], inp["W_lin"], inp["gates"], cfg.T)
+    np.testing.assert_array_equal(ulysses.ulysses_forward(*args, fwd=fwd).numpy(),
+                                  fwd(*args).numpy())
+
+
+def test_head_split_must_divide():
+    from softmax_attention_video_chunk_b200 import ulysses
+    with pytest.raises(ValueError):
+        ulysses.head_slice(3, 0, 4)
+    assert ulysses.head_slice(4, 3, 8) == slice(6, 8)
