@@ -406,7 +406,8 @@ def run_ours(args, cfg):
                                              (2 if prep_ms is not None else 0))
         if tq_ms is not None:
             line["stages_ms"]["text_rows"] = round(tq_ms, 4)
-            line["gpu_launches"] += args.steps * 2  # V^T conversion + text-row Softmax
+            # V^T conversion, text-row Softmax split over key shares, combine
+            line["gpu_launches"] += args.steps * 3
         if prep_ms is not None:
             es = 2 if cfg.dtype == "bf16" else 4
             prep_bytes = 6 * cfg.B * cfg.L * cfg.H * cfg.d * es  # read q, k, v; write 3

@@ -128,7 +128,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                const __grid_constant__ CUtensorMap map_tvt, int n_text, Geo geo, int B, int H,
                float scale_log2, const __nv_bfloat16* __restrict__ gates,
                __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status,
-               int n_qtext) {
+               int n_qtext, int kv_split, float* __restrict__ ml) {
   constexpr int BM = 128, NS = 2;
   constexpr int QT = BM * D * 2;   // bytes of a Q tile
   constexpr int KT = kBK * D * 2;  // bytes of a K tile
@@ -154,7 +154,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = B * H;
-  const int pair = blockIdx.x / BH, bh = blockIdx.x % BH;
+  // kv_split > 1 (text rows only): CTA `split` of a row pair walks its share
+  // of the key tiles and writes a partial result (o normalised by its own sum,
+  // plus the running max and sum) for a combine pass
+  const int pq = blockIdx.x / BH, bh = blockIdx.x % BH;
+  const int pair = pq / kv_split, split = pq % kv_split;
   const int b = bh / H, h = bh % H;
   QGroup g;
   int row0;
@@ -170,7 +174,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
   const int row_end = g.row0 + g.nrows;
   const bool has1 = row0 + BM < row_end;
   const int n_video = kv_count(g);
-  const int n_kv = n_video + (n_text + kBK - 1) / kBK;
+  const int n_all = n_video + (n_text + kBK - 1) / kBK;
+  const int kv0 = (int)((long long)n_all * split / kv_split);  // this CTA: tiles kv0 ..
+  const int n_kv = (int)((long long)n_all * (split + 1) / kv_split) - kv0;
   const int L = geo.T * geo.N;
 
   if (threadIdx.x == 0) {
@@ -220,7 +226,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         if (use > 0 && !wait_bar(kv_empty + st, (use - 1) & 1, ab)) break;
         int k0, lo, hi;
         bool text;
-        kv_tile_all(g, n_video, n_text, i, k0, lo, hi, text);
+        kv_tile_all(g, n_video, n_text, kv0 + i, k0, lo, hi, text);
         const CUtensorMap* mk = text ? &map_tk : &map_k;
         const CUtensorMap* mv = text ? &map_tvt : &map_vt;
         ptx::mbar_arrive_expect_tx(k_full + st, KT);
@@ -311,7 +317,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
       for (int i = 0; i < n_kv; ++i) {
         int k0, lo, hi;
         bool text;
-        kv_tile_all(g, n_video, n_text, i, k0, lo, hi, text);
+        kv_tile_all(g, n_video, n_text, kv0 + i, k0, lo, hi, text);
         if (!(ok = wait_bar(s_full + j, i & 1, ab))) break;
         ptx::tc_fence_after();
         // pass 1: row maximum (all four 32-column loads in flight at once)
@@ -447,6 +453,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const float inv = 1.f / l_sum;
         const size_t tok = (size_t)b * (n_qtext > 0 ? n_qtext : L) + row;
         bool bad = false;
+        float* o_out = o_s;
+        if (kv_split > 1) {  // partial result of this key share
+          const size_t rows_all = (size_t)B * n_qtext * H;
+          o_out = o_s + (size_t)split * rows_all * D;
+          if (valid) {
+            float* mlp = ml + ((size_t)split * rows_all + tok * H + h) * 2;
+            mlp[0] = m_used;
+            mlp[1] = l_sum;
+          }
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -473,7 +489,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
               xp[v4] = outv;
             }
           } else {
-            float4* op = reinterpret_cast<float4*>(o_s + (tok * H + h) * D + 32 * c);
+            float4* op = reinterpret_cast<float4*>(o_out + (tok * H + h) * D + 32 * c);
 #pragma unroll
             for (int v4 = 0; v4 < 8; ++v4)
               op[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv, __uint_as_float(o[4 * v4 + 1]) * inv,
@@ -488,6 +504,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+// Text rows split over key shares: o = sum_s w_s o_s / sum_s w_s with
+// w_s = l_s 2^(m_s - max_s m_s) (o_s normalised by its own sum l_s, m_s the
+// running maximum in log2 units).  One warp per (token, head) row.
+template <int D>
+__global__ void __launch_bounds__(256)
+combine_splits_kernel(const float* __restrict__ part, const float* __restrict__ ml,
+                      float* __restrict__ out, size_t rows, int S) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[((size_t)s * rows + r) * 2]);
+  float W = 0.f, acc[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float* m2 = ml + ((size_t)s * rows + r) * 2;
+    const float w = m2[1] * exp2f(m2[0] - M);
+    W += w;
+    const float* p = part + ((size_t)s * rows + r) * D + lane * CPL;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) acc[i] = fmaf(w, p[i], acc[i]);
+  }
+  const float inv = 1.f / W;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) out[r * D + lane * CPL + i] = acc[i] * inv;
 }
 
 // --------------------------------------------------------------------------
@@ -542,7 +587,9 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
       return cudaErrorInvalidValue;
   }
   Geo geo{t.T, t.N, t.C, t.R};
-  const int pairs = n_qtext > 0 ? (n_qtext + 255) / 256 : count_tiles(geo, 256);
+  const int kv_split = (n_qtext > 0 && t.part != nullptr && t.kv_split > 1) ? t.kv_split : 1;
+  const int pairs =
+      (n_qtext > 0 ? (n_qtext + 255) / 256 : count_tiles(geo, 256)) * kv_split;
   const size_t sm = 1024 + 2 * (128 * D * 2) + 2 * 2 * (128 * D * 2) + 256;
   auto kern = attn_tc_kernel<D, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -551,8 +598,16 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
   const unsigned grid = (unsigned)pairs * (unsigned)(t.B * t.H);
   kern<<<grid, 320, sm, st>>>(mq, mk, mv, mtk, mtv, t.n_text_keys, geo, t.B, t.H, scale_log2,
                               FUSED ? (const __nv_bfloat16*)f->gates : nullptr,
-                              FUSED ? f->x : nullptr, o_s, t.status, n_qtext);
-  return cudaGetLastError();
+                              FUSED ? f->x : nullptr, kv_split > 1 ? t.part : o_s, t.status,
+                              n_qtext, kv_split, t.ml);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (kv_split > 1) {
+    const size_t rows = (size_t)t.B * n_qtext * t.H;
+    combine_splits_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(t.part, t.ml, o_s, rows,
+                                                                           kv_split);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_attn_tc(const TcAttnArgs& t, const TcFwdArgs* f, float* o_s, cudaStream_t st) {

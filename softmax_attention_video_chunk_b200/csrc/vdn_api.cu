@@ -102,6 +102,8 @@ vdn_status boundary_states_impl(const vdn_params* p, const void* k, const void* 
                                 const void* text_v, float* F, float* G, void* workspace,
                                 vdn_stream_t stream);
 
+int sm_count();
+
 static vdn_status validate_prep(const vdn_prep_params* p) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;
   if (p->B < 1 || p->H < 1 || p->T < 1 || p->grid_h < 1 || p->grid_w < 1) return VDN_ERR_SHAPE;
@@ -475,6 +477,21 @@ vdn_status vdn_text_query_attn(const vdn_params* p, const void* text_q, const vo
   a.text_q = text_q;
   if (use_tc(pt)) {
     TcAttnArgs t = tc_attn_args(pt, a, ws + w.vt, (int*)(ws + w.status));
+    // split the keys of the few text-row CTAs until the grid covers the GPU
+    // twice; the partial results live in the (here unused) operand region x
+    const int tiles = (int)((pt.T * (size_t)pt.N + 127) / 128 + (pt.n_text + 127) / 128);
+    const long long base = (long long)((pt.n_text + 255) / 256) * pt.B * pt.H;
+    int split = (int)((2LL * sm_count() + base - 1) / base);
+    split = split < 1 ? 1 : (split > 16 ? 16 : split);
+    if (split > tiles / 2) split = tiles / 2 > 1 ? tiles / 2 : 1;
+    const size_t rows = (size_t)pt.B * pt.n_text * pt.H;
+    while (split > 1 && (size_t)split * rows * (pt.d_k + 2) * sizeof(float) > w.total - w.x)
+      --split;
+    if (split > 1) {
+      t.kv_split = split;
+      t.part = (float*)(ws + w.x);
+      t.ml = t.part + (size_t)split * rows * pt.d_k;
+    }
     VDN_CUDA(launch_convert_v(t, st));
     VDN_CUDA(launch_attn_tc(t, nullptr, o_text, st));
   } else {

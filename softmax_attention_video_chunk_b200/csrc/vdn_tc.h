@@ -24,6 +24,9 @@ struct TcAttnArgs {
   const void *text_k, *text_v;  // bf16 [B, n_text, H, D]
   __half* vt_text;        // fp16 [B*H][D][ntp], text V transposed
   const void* text_q = nullptr;  // bf16 [B, n_text, H, D]: text queries (dense rows)
+  int kv_split = 1;              // text rows: key tiles split over this many CTAs
+  float* part = nullptr;         // [kv_split][B*n_text*H][D] partial outputs
+  float* ml = nullptr;           // [kv_split][B*n_text*H][2] running max and sum
 };
 
 struct TcFwdArgs {
