@@ -175,3 +175,28 @@ def test_split_forward_requires_linear_inputs():
     rc = L.vdn_hybrid_attn_fwd_split(ctypes.byref(p), *ptr, ctypes.c_void_p(0x80000),
                                      1 << 40, None, None)
     assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"
+
+
+def test_text_query_attn_validates_before_launch():
+    L = vdn.lib()
+    ptr = [ctypes.c_void_p(0x1000 * (i + 1)) for i in range(6)]  # text_q k v text_k text_v o_text
+    p = vdn.make_params(1, 2, 15, 16, 64, 0, "bf16")  # no text tokens
+    rc = L.vdn_text_query_attn(ctypes.byref(p), *ptr, ctypes.c_void_p(0x80000), 1 << 40, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_SHAPE"
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    bad = list(ptr)
+    bad[0] = ctypes.c_void_p(0)  # text_q missing
+    rc = L.vdn_text_query_attn(ctypes.byref(p), *bad, ctypes.c_void_p(0x80000), 1 << 40, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"
+    # the workspace must hold the text tokens' V^T (sized as with VDN_FLAG_TEXT_SOFTMAX)
+    need = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", text_softmax=True))
+    assert need > vdn.workspace_bytes(p)
+    rc = L.vdn_text_query_attn(ctypes.byref(p), *ptr, ctypes.c_void_p(0x80000),
+                               vdn.workspace_bytes(p), None)
+    assert vdn.STATUS[rc] == "VDN_ERR_WORKSPACE"
+
+
+def test_frozen_state_flag_is_accepted():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", frozen_state=True)
+    assert p.flags & vdn.FLAG_FROZEN_STATE
+    assert vdn.workspace_bytes(p) == vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8))
