@@ -153,10 +153,10 @@ def blas_threads():
 def oracle_sample(cfg, inp):
     """A fixed, bounded sample of the workload for the CPU oracle (about 10 s
     on 16 host cores at 768p): 4 query tokens of the anchor frame 0 and 4 of
-    each of five mid-clip frames in different chunks (12, 27, 37, 52, 62), with
+    each of seven frames in different chunks (7, 12, 27, 37, 52, 62, 72), with
     all heads, including the frame-by-frame VDA recurrence each chunk needs."""
     import numpy as np
-    frames = sorted({0} | {min(cfg.T - 2, f) for f in (12, 27, 37, 52, 62)})
+    frames = sorted({0} | {min(cfg.T - 2, f) for f in (7, 12, 27, 37, 52, 62, 72)})
     pick = (0, cfg.N // 3, 2 * cfg.N // 3, cfg.N - 1)
     return np.array([t * cfg.N + n for t in frames for n in pick])
 
