@@ -238,6 +238,43 @@ def test_ulysses_one_rank_runs_the_library_forward():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("simt", [False, True])
+def test_poisoned_workspace_is_never_read_before_written(simt):
+    """Every byte of scratch the path reads is written first by the same call:
+    a workspace filled with NaN bytes (0xFF) gives bit-identical, finite
+    results to a zero-filled one (forward with text keys and per-token gates,
+    the two branches, the boundary states and the text rows)."""
+    cfg = _edge_cfg(dict(T=13, N=72, n_text=40))
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0), beta_per_token=True)
+    d = to_dev(inp)
+    tq = make_text_queries(cfg).cuda()
+    p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], text_softmax=True,
+                       beta_per_token=True, simt=simt)
+
+    def run(fill):
+        ws = vdn.alloc_workspace(p)
+        ws.fill_(fill)
+        out = _fwd(d, cfg, params=p, workspace=ws)
+        ws.fill_(fill)
+        o_s, o_l = vdn.hybrid_attn_branches(d["q"], d["k"], d["v"], d["beta"], d["text_k"],
+                                            d["text_v"], cfg.T, alpha=d["alpha"], workspace=ws,
+                                            params=p)
+        ws.fill_(fill)
+        F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
+                                       alpha=d["alpha"], workspace=ws, params=p)
+        ws.fill_(fill)
+        ot = vdn.text_query_attn(tq, d["k"], d["v"], d["text_k"], d["text_v"], cfg.T,
+                                 workspace=ws, params=p)
+        torch.cuda.synchronize()
+        assert vdn.STATUS[vdn.device_status(p, ws)] == "VDN_OK"
+        return [out, o_s, o_l, F, G, ot]
+
+    clean, poisoned = run(0), run(255)
+    for a, b in zip(clean, poisoned):
+        assert torch.isfinite(b).all()
+        assert torch.equal(a, b)
+
+
 def test_wide_scores_rescale_path():
     """Scores spanning many octaves (q scaled up): the running-max rescale of
     the tensor-core kernel is exercised."""
