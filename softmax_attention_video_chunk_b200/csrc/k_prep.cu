@@ -54,7 +54,6 @@ constexpr int kTaps = 5;  // temporal taps
 #endif
 constexpr int kPos = VDN_PREP_POS;  // grid columns per warp
 
-
 // A lane's CPL channels as packed FP32 pairs (fma.rn.f32x2); for CPL = 1 the
 // upper half of the single pair is unused.
 template <int CPL>

@@ -114,6 +114,8 @@ static vdn_status validate_prep(const vdn_prep_params* p) {
   // the TMA frame coordinate and the grid extents are 32-bit
   if ((long long)p->B * p->T > (1ll << 30) || (long long)p->grid_h * p->grid_w > (1ll << 30))
     return VDN_ERR_SHAPE;
+  // launch grid: y = grid rows, z = (batch, head, K or V)
+  if (p->grid_h > 65535 || 2LL * p->B * p->H > 65535) return VDN_ERR_SHAPE;
   return VDN_OK;
 }
 

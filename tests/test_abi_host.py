@@ -136,7 +136,8 @@ def test_prep_params_defaults_and_validation():
     for field, value, code in [("d", 96, "VDN_ERR_UNSUPPORTED"), ("spatial_taps", 5, "VDN_ERR_UNSUPPORTED"),
                                ("temporal_taps", 3, "VDN_ERR_UNSUPPORTED"), ("grid_w", 0, "VDN_ERR_SHAPE"),
                                ("T", 0, "VDN_ERR_SHAPE"), ("dtype", 4, "VDN_ERR_DTYPE"),
-                               ("l2_eps", -1.0, "VDN_ERR_INVALID_ARG")]:
+                               ("l2_eps", -1.0, "VDN_ERR_INVALID_ARG"),
+                               ("grid_h", 70000, "VDN_ERR_SHAPE"), ("H", 40000, "VDN_ERR_SHAPE")]:
         q = vdn.make_prep_params(1, 2, 4, 3, 5, 64, "bf16")
         setattr(q, field, value)
         ptrs = [0x1000 * (i + 1) for i in range(10)]
