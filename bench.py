@@ -69,9 +69,9 @@ def work_model(cfg, out_bytes=4, text_keys=False):
 
 # DRAM bytes (read + write) of one attn_tc_kernel launch, from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum) of the 4-head copy of the
-# 768p workload: 964.0 MB + 115.8 MB, scaled by the head count (the launch is
+# 768p workload: 1001.1 MB + 113.2 MB, scaled by the head count (the launch is
 # one independent problem per head).  None for any other workload.
-ATTN_TRAFFIC_PER_HEAD = (963.955968e6 + 115.819008e6) / 4
+ATTN_TRAFFIC_PER_HEAD = (1001.119e6 + 113.169152e6) / 4
 ATTN_TRAFFIC_SHAPES = {(75, 1536, 128)}
 
 
