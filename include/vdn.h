@@ -301,17 +301,31 @@ VDN_API vdn_status vdn_vda_boundary_states(const vdn_params *p, const void *k, c
  *    VDN_ERR_WORKSPACE.  The scratch is about
  *    4 * d*d * B*H * (2*(T+1) + 6*ceil(T/chunk) + 2) bytes: e.g. B*H = 8,
  *    T = 40, d = 64 needs 17 MiB and fits; the 768p workload does not.
- *  - The first call on a device looks up the array's device address (with that
- *    device current); make that first call before any stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (a table read once the library is loaded there; nothing is cached, so a
+ *    context destroyed and re-created by cudaDeviceReset is handled).  The
+ *    first call on a device may load the library's module there: make it
+ *    before any stream capture.
  *  - All calls share the one array and it keeps the last call's contents:
  *    calls that overlap on the GPU (unordered streams or threads) race.  Order
- *    them on one stream.  The device status word is cleared by each call.
+ *    them on one stream.
+ *  - Device-side conditions (VDN_ERR_TIMEOUT, VDN_ERR_RANGE) go to a status
+ *    word at the start of the array, cleared when each call starts: read it
+ *    with vdn_noalloc_device_status.
  *  - Other conventions as vdn_vda_boundary_states; no workspace arguments. */
 VDN_API vdn_status vdn_vda_boundary_states_noalloc(const vdn_params *p, const void *k,
                                                    const void *v, const float *beta,
                                                    const float *alpha, const void *text_k,
                                                    const void *text_v, float *F, float *G,
                                                    vdn_stream_t stream);
+
+/* Status of the last vdn_vda_boundary_states_noalloc call on the current
+ * device: synchronises `stream`, then reads and clears the status word in the
+ * library's static array (VDN_OK, VDN_ERR_TIMEOUT or VDN_ERR_RANGE).  Like
+ * that entry point it has no counterpart in the paper and allocates nothing.
+ * A status word is shared by every no-allocation call on the device: read it
+ * after the call whose status you want, before the next one is enqueued. */
+VDN_API vdn_status vdn_noalloc_device_status(vdn_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * the last compute call on this workspace left (VDN_OK, VDN_ERR_TIMEOUT or
@@ -333,6 +347,16 @@ VDN_API vdn_status vdn_device_status(const vdn_params *p, void *workspace, vdn_s
  *  - The GPU context stays usable; later calls run normally. */
 VDN_API vdn_status vdn_selftest_bounded_wait(void *workspace, unsigned int limit_us,
                                              vdn_stream_t stream);
+
+/* Self-test of the exponential that the tensor-core Softmax kernel evaluates
+ * on the FMA pipe for a share of its P = 2^x values (to relieve the MUFU
+ * pipe): y[i] = 2^x[i] by a Cody-Waite split x = n + f, n = round(x), and a
+ * degree-4 minimax polynomial for 2^f (relative error below 3e-6), with x
+ * clamped below at -125 (so every x <= -125 gives 2^-125, which is zero once
+ * rounded to the fp16 P operand).  Valid for x <= 64.
+ *  - x, y: float32 device arrays of n elements (y may be x); asynchronous on
+ *    `stream`; VDN_ERR_INVALID_ARG for NULL pointers. */
+VDN_API vdn_status vdn_selftest_exp2(const float *x, float *y, size_t n, vdn_stream_t stream);
 
 #ifdef __cplusplus
 }

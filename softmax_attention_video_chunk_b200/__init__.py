@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_vda_boundary_states.argtypes = [PP] + [_P] * 9 + [ctypes.c_size_t, _P]
         L.vdn_vda_boundary_states_noalloc.restype = ctypes.c_int
         L.vdn_vda_boundary_states_noalloc.argtypes = [PP] + [_P] * 8 + [_P]
+        L.vdn_noalloc_device_status.restype = ctypes.c_int
+        L.vdn_noalloc_device_status.argtypes = [_P]
         L.vdn_device_status.restype = ctypes.c_int
         L.vdn_device_status.argtypes = [PP, _P, _P]
         L.vdn_hybrid_attn_fwd_split.restype = ctypes.c_int
@@ -107,6 +109,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_text_query_attn.argtypes = [PP] + [_P] * 7 + [ctypes.c_size_t, _P]
         L.vdn_selftest_bounded_wait.restype = ctypes.c_int
         L.vdn_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint, _P]
+        L.vdn_selftest_exp2.restype = ctypes.c_int
+        L.vdn_selftest_exp2.argtypes = [_P, _P, ctypes.c_size_t, _P]
         _lib = L
     return _lib
 
@@ -363,6 +367,12 @@ def vda_boundary_states_noalloc(k, v, beta, text_k, text_v, T, *, alpha=None, st
     return F, G
 
 
+def noalloc_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status word of the last
+    vda_boundary_states_noalloc call on the current device."""
+    return lib().vdn_noalloc_device_status(_stream(stream))
+
+
 def device_status(p: Optional[VdnParams], workspace, stream=None) -> int:
     """Synchronise and return (and clear) the device status of the last call
     (``p`` may be None, e.g. for the VDA-Prep workspace)."""
@@ -373,6 +383,19 @@ def device_status(p: Optional[VdnParams], workspace, stream=None) -> int:
 def selftest_bounded_wait(workspace, limit_us: int, stream=None) -> int:
     """Enqueue the bounded-wait self-test (a wait that nothing satisfies)."""
     return lib().vdn_selftest_bounded_wait(_ptr(workspace), int(limit_us), _stream(stream))
+
+
+def selftest_exp2(x, stream=None):
+    """2^x (float32 device tensor) through the Softmax kernel's FMA-pipe
+    exponential (vdn_selftest_exp2)."""
+    import torch
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    y = torch.empty_like(x)
+    rc = lib().vdn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_selftest_exp2")
+    return y
 
 
 def use_tc_params(p: VdnParams) -> bool:

@@ -12,10 +12,9 @@
 // The array is VDN_NOALLOC_SCRATCH_BYTES large; every GPU that loads the
 // library holds it until the process exits.  All calls share it: calls that
 // overlap on the GPU (different streams or threads without ordering) race on
-// it.  Its status word is cleared by each call; every other byte the path reads
-// is written first by the same call.
-#include <mutex>
-
+// it.  Its first bytes hold the device status word of the last call (cleared
+// when each call starts; read it with vdn_noalloc_device_status); every other
+// byte the path reads is written first by the same call.
 #include "vdn_common.cuh"
 #include "vdn_kernels.h"
 
@@ -28,27 +27,19 @@ vdn_status boundary_states_impl(const vdn_params* p, const void* k, const void* 
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[VDN_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch, looked up once per device with that
-// device current (the host-side name is only a stand-in, not a device pointer).
+// Device address of g_noalloc_scratch on the current device (the host-side
+// name is only a stand-in, not a device pointer).  Looked up on every call,
+// with the caller's device current, so that a context torn down and made
+// again (cudaDeviceReset) never leaves a stale address behind; the lookup is a
+// table read once the library's module is loaded on that device.
 static void* scratch_address(vdn_status* err) {
-  static std::mutex mu;
-  static void* addr[128] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
     *err = VDN_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      *err = VDN_ERR_CUDA;
-      return nullptr;
-    }
-    addr[dev] = p;
-  }
   *err = VDN_OK;
-  return addr[dev];
+  return p;
 }
 }  // namespace vdn
 
@@ -65,4 +56,18 @@ extern "C" vdn_status vdn_vda_boundary_states_noalloc(const vdn_params* p, const
   void* scratch = vdn::scratch_address(&err);
   if (scratch == nullptr) return err;
   return vdn::boundary_states_impl(p, k, v, beta, alpha, text_k, text_v, F, G, scratch, stream);
+}
+
+extern "C" vdn_status vdn_noalloc_device_status(vdn_stream_t stream) {
+  vdn_status err = VDN_OK;
+  void* scratch = vdn::scratch_address(&err);
+  if (scratch == nullptr) return err;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return VDN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (cudaMemset(scratch, 0, sizeof(int)) != cudaSuccess) return VDN_ERR_CUDA;
+  if (word & vdn::kDevTimeout) return VDN_ERR_TIMEOUT;
+  if (word & vdn::kDevRange) return VDN_ERR_RANGE;
+  return VDN_OK;
 }

@@ -48,9 +48,32 @@ selftest_wait_kernel(int* __restrict__ status, unsigned long long limit_ns) {
   }
 }
 
+// y = 2^x through the FMA-pipe polynomial exponential the Softmax kernel
+// uses for a share of its P values (ptx::exp2_poly2), two lanes at a time.
+__global__ void __launch_bounds__(256) selftest_exp2_kernel(const float* __restrict__ x,
+                                                            float* __restrict__ y, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x * 2;
+  for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 2; i < n; i += stride) {
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+    float y0, y1;
+    ptx::f2_unpack(ptx::exp2_poly2(ptx::f2_pack(x0, x1)), y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+  }
+}
+
 }  // namespace vdn
 
 extern "C" {
+
+vdn_status vdn_selftest_exp2(const float* x, float* y, size_t n, vdn_stream_t stream) {
+  if (x == nullptr || y == nullptr) return VDN_ERR_INVALID_ARG;
+  if (n == 0) return VDN_OK;
+  const size_t blocks = (n + 511) / 512;
+  vdn::selftest_exp2_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0,
+                              (cudaStream_t)stream>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
 
 vdn_status vdn_selftest_bounded_wait(void* workspace, unsigned int limit_us,
                                      vdn_stream_t stream) {

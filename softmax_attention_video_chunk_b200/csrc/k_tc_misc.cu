@@ -15,6 +15,9 @@
 // implementation ("VDA-Gather", "VDA-Epilogue" fused kernels).
 #include <math.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "tc_ptx.cuh"
 #include "vdn_common.cuh"
 #include "vdn_tc.h"
@@ -29,18 +32,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once per process; std::call_once makes the first concurrent calls
+// from several host threads safe.
 static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = (EncodeTiledFn)p;
-  }
+  });
   return fn;
 }
 
@@ -391,17 +395,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
+// SM count of the current device (the per-device attribute cache; atomic
+// entries, so concurrent first calls are safe).
 int sm_count() {
-  static int cached[128] = {0};
+  static std::atomic<int> cached[128];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 cudaError_t launch_gemm_tc(const TcFwdArgs& f, cudaStream_t st) {

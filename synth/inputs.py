@@ -21,6 +21,9 @@ standard workloads (alpha == 1); ``alpha_range`` draws alpha ~ U[lo, hi]
 per (b, h, frame, channel) as an extra draw after the gates;
 ``beta_per_token`` then draws one write gate per token,
 sigmoid(N(0, 1)) [B, H, n_text + L] (text tokens first), replacing beta.
+``gates="random"`` replaces the constant gates with independent per-element
+draws g_s, g_l = sigmoid(N(0, 1)) [B, L, H, d] each (Softmax gate first), taken
+after every other draw so that nothing else changes.
 
 L = T * N and token index = t * N + n (frame-major, token-minor).
 """
@@ -90,7 +93,7 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 
 def make_inputs(cfg: Config, *, alpha_range: Optional[tuple] = None,
                 beta_override: Optional[torch.Tensor] = None, beta_per_token: bool = False,
-                device: str = "cpu") -> dict:
+                gates: str = "const", device: str = "cpu") -> dict:
     """Draw one workload.  Returns torch tensors in the workload dtype
     (beta, alpha always float32) on ``device``.
 
@@ -128,6 +131,13 @@ def make_inputs(cfg: Config, *, alpha_range: Optional[tuple] = None,
         out["alpha"] = None
     if beta_per_token:
         out["beta"] = torch.sigmoid(randn(B, H, cfg.n_text + L))
+    if gates == "random":
+        g_s = torch.sigmoid(randn(B, L, H, d))
+        g_l = torch.sigmoid(randn(B, L, H, d))
+        out["gates"] = torch.stack([g_s, g_l]).to(dt)
+        del g_s, g_l
+    elif gates != "const":
+        raise ValueError(f"gates must be 'const' or 'random', not {gates!r}")
     if device != "cpu":
         out = {k: (v.to(device) if v is not None else None) for k, v in out.items()}
     return out

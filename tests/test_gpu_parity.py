@@ -38,10 +38,11 @@ def _branches(d, cfg, **kw):
 # full comparison on small workloads
 # ----------------------------------------------------------------------------
 
+@pytest.mark.parametrize("gates", ["const", "random"])
 @pytest.mark.parametrize("simt", [False, True])
-def test_tiny_f32_full(simt):
+def test_tiny_f32_full(simt, gates):
     cfg = CONFIGS["tiny_f32"]
-    inp = make_inputs(cfg)
+    inp = make_inputs(cfg, gates=gates)
     d = to_dev(inp)
     out = _fwd(d, cfg, simt=simt)
     o_s, o_l = _branches(d, cfg, simt=simt)
@@ -58,10 +59,11 @@ def test_tiny_f32_full(simt):
     assert rel_err(G.double().cpu(), Go) <= 1e-5
 
 
+@pytest.mark.parametrize("gates", ["const", "random"])
 @pytest.mark.parametrize("simt", [False, True])
-def test_small_bf16_full(simt):
+def test_small_bf16_full(simt, gates):
     cfg = CONFIGS["small_bf16"]
-    inp = make_inputs(cfg)
+    inp = make_inputs(cfg, gates=gates)
     d = to_dev(inp)
     out = _fwd(d, cfg, simt=simt)
     o_s, o_l = _branches(d, cfg, simt=simt)
@@ -70,7 +72,8 @@ def test_small_bf16_full(simt):
     e_out = rel_err(out.double().cpu(), want)
     e_s = rel_err(o_s.double().cpu(), ws_)
     e_l = rel_err(o_l.double().cpu(), wl_)
-    print(f"small_bf16 simt={simt}: out {e_out:.2e} o_soft {e_s:.2e} o_lin {e_l:.2e}")
+    print(f"small_bf16 simt={simt} gates={gates}: out {e_out:.2e} o_soft {e_s:.2e} "
+          f"o_lin {e_l:.2e}")
     assert e_out <= TOL_OUT["bf16"]
     assert e_s <= 2e-3
     assert e_l <= 1e-4
@@ -95,6 +98,11 @@ EDGE = [
      dict(beta_per_token=True), dict(beta_per_token=True)),
     ("d128", dict(T=11, N=136, d=128, H=2), {}, {}),
     ("d32", dict(T=11, N=40, d=32, H=3), {}, {}),
+    # independent per-element gates of the two branches (sigmoid(N(0,1)))
+    ("gates_d128", dict(T=11, N=136, d=128, H=2), dict(gates="random"), {}),
+    ("gates_ragged_N", dict(T=13, N=37, d=64, H=3), dict(gates="random"), {}),
+    ("gates_text_softmax_d128", dict(T=9, N=130, d=128, H=2, n_text=77),
+     dict(gates="random", alpha_range=(0.9, 1.0)), dict(text_softmax=True)),
 ]
 
 
@@ -353,8 +361,8 @@ def test_bounded_wait_expires_into_status():
 # full-size workloads, sampled rows
 # ----------------------------------------------------------------------------
 
-def _sampled(cfg, rows, bsel, chunk=None, alpha_range=None, **kw):
-    inp = make_inputs(cfg, alpha_range=alpha_range)
+def _sampled(cfg, rows, bsel, chunk=None, alpha_range=None, gates="const", **kw):
+    inp = make_inputs(cfg, alpha_range=alpha_range, gates=gates)
     d = to_dev(inp)
     c = cfg.chunk if chunk is None else chunk
     out = vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
@@ -373,6 +381,27 @@ def test_768p_sampled():
     rows = sample_rows(cfg, per_frame=3)
     e = _sampled(cfg, rows, None)
     print(f"768p sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_768p_random_gates_sampled():
+    """The 768p workload with independent per-element gates g_s, g_l ~
+    sigmoid(N(0, 1)): the fused epilogues of the Softmax and readout kernels
+    read their own gate at the (token, head, channel) of each output."""
+    cfg = CONFIGS["768p_bf16"]
+    rows = sample_rows(cfg, per_frame=2, chunks=[0, 1, 7, 13, 14])
+    e = _sampled(cfg, rows, None, gates="random")
+    print(f"768p random gates sampled ({len(rows)} rows): {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_batched_random_gates_sampled():
+    """Batched clips with random per-element gates: gate rows of batch items
+    other than the first are indexed with the batch offset."""
+    cfg = CONFIGS["batched_bf16"]
+    rows = sample_rows(cfg, per_frame=2)
+    e = _sampled(cfg, rows, [5, 15], gates="random")
+    print(f"batched random gates sampled: {e:.2e}")
     assert e <= TOL_OUT["bf16"]
 
 

@@ -518,3 +518,114 @@ def test_per_token_beta_constant_equals_per_frame():
     a = O.linear_branch(q, k, v, beta, tk, tv, T, N, 5, 1, alpha=alpha)
     b = O.linear_branch(q, k, v, per_tok, tk, tv, T, N, 5, 1, alpha=alpha, beta_per_token=True)
     np.testing.assert_allclose(b, a, rtol=1e-11, atol=1e-12)
+
+
+# --- Gate routing of the whole forward ---------------------------------------
+
+def _routing_case():
+    from synth import CONFIGS, make_inputs
+    cfg = CONFIGS["tiny_f32"].replace(T=7, N=6, H=2, d=32, n_text=5, seed=41)
+    inp = make_inputs(cfg, gates="random")
+    a = {k: (None if v is None else O._to_np(v)) for k, v in inp.items()}
+    return cfg, inp, a
+
+
+def _loop_projection(x, W):
+    """out[b, r, :] = sum_h sum_c x[b, r, h, c] * W[h * d + c, :], written as
+    explicit loops over heads and channels (no reshape)."""
+    B, R, H, d = x.shape
+    out = np.zeros((B, R, W.shape[1]))
+    for b in range(B):
+        for r in range(R):
+            for h in range(H):
+                for c in range(d):
+                    out[b, r] += x[b, r, h, c] * W[h * d + c]
+    return out
+
+
+def _check_routing(fwd):
+    """Raises AssertionError unless ``fwd`` (the oracle's hybrid_forward, or a
+    variant of it) routes each gate to its own branch and projection."""
+    cfg, inp, a = _routing_case()
+    T, N = cfg.T, cfg.N
+    o_s = O.softmax_branch(a["q"], a["k"], a["v"], T, N, cfg.chunk, cfg.window_radius)
+    o_l = O.linear_branch(a["q"], a["k"], a["v"], a["beta"], a["text_k"], a["text_v"], T, N,
+                          cfg.chunk, cfg.window_radius)
+    g_s, g_l = a["gates"][0], a["gates"][1]
+    assert np.std(g_s) > 0.05 and np.max(np.abs(g_s - g_l)) > 0.3  # two different gates
+    soft_half = _loop_projection(g_s * o_s, a["W_soft"])
+    ms = np.mean(o_l * o_l, axis=-1, keepdims=True)
+    lin_half = _loop_projection(g_l * o_l / np.sqrt(ms + 1e-6), a["W_lin"])
+
+    only_soft = dict(inp)
+    only_soft["gates"] = inp["gates"].clone()
+    only_soft["gates"][1] = 0
+    out, _, _ = fwd(only_soft, T, N, cfg.chunk, cfg.window_radius)
+    np.testing.assert_allclose(out, soft_half, rtol=1e-10, atol=1e-12)
+
+    only_lin = dict(inp)
+    only_lin["gates"] = inp["gates"].clone()
+    only_lin["gates"][0] = 0
+    out, _, _ = fwd(only_lin, T, N, cfg.chunk, cfg.window_radius)
+    np.testing.assert_allclose(out, lin_half, rtol=1e-10, atol=1e-12)
+
+    out, _, _ = fwd(inp, T, N, cfg.chunk, cfg.window_radius)
+    np.testing.assert_allclose(out, soft_half + lin_half, rtol=1e-10, atol=1e-12)
+    # the gates are not interchangeable: swapping them moves the output
+    swapped = dict(inp)
+    swapped["gates"] = inp["gates"].flip(0)
+    out_sw, _, _ = fwd(swapped, T, N, cfg.chunk, cfg.window_radius)
+    assert np.max(np.abs(out_sw - out)) > 1e-2 * np.sqrt(np.mean(out ** 2))
+
+
+def test_forward_routes_each_gate_to_its_own_branch_and_projection():
+    """The pages' output stage: the Softmax readout is gated by its own sigmoid
+    gate and projected by its own matrix; the linear readout is RMS-normalised,
+    gated by the second gate and projected by the second matrix; the two are
+    added.  With g_l = 0 the forward is the Softmax half alone, with g_s = 0 the
+    linear half alone (each rebuilt here with per-head, per-channel loops), and
+    with both gates random the forward is their sum."""
+    _check_routing(O.hybrid_forward)
+
+
+@pytest.mark.parametrize("mistake", ["swap_gates", "swap_projections", "transpose_gate"])
+def test_routing_pin_catches_planted_mistakes(monkeypatch, mistake):
+    """The routing pin fails on an oracle with a planted mistake in its output
+    stage (patched here, on the CPU): gates swapped between the branches,
+    projections swapped, or the gate's head and channel axes transposed."""
+    real = O.output_projection
+
+    def planted(o_s, o_l, g_s, g_l, W_soft, W_lin, eps=1e-6):
+        if mistake == "swap_gates":
+            return real(o_s, o_l, g_l, g_s, W_soft, W_lin, eps)
+        if mistake == "swap_projections":
+            return real(o_s, o_l, g_s, g_l, W_lin, W_soft, eps)
+        gs = np.asarray(g_s, np.float64)
+        B, R, H, d = gs.shape
+        gs = gs.reshape(B, R, H * d).reshape(B, R, d, H).swapaxes(-1, -2)
+        return real(o_s, o_l, gs, g_l, W_soft, W_lin, eps)
+
+    monkeypatch.setattr(O, "output_projection", planted)
+    with pytest.raises(AssertionError):
+        _check_routing(O.hybrid_forward)
+
+
+def test_gate_rows_follow_the_sampled_query_rows():
+    """Forward on a subset of query rows equals the same rows of the full
+    forward, with random per-element gates (the gate rows follow the rows)."""
+    cfg, inp, _ = _routing_case()
+    full, _, _ = O.hybrid_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    rows = np.array([0, 5, 6, 17, 23, cfg.T * cfg.N - 1])
+    part, _, _ = O.hybrid_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius, rows=rows)
+    np.testing.assert_allclose(part, full[:, rows], rtol=1e-12, atol=1e-13)
+
+
+def test_random_gates_leave_every_other_draw_unchanged():
+    from synth import CONFIGS, make_inputs
+    cfg = CONFIGS["tiny_f32"]
+    a, b = make_inputs(cfg), make_inputs(cfg, gates="random", alpha_range=(0.9, 1.0))
+    for k in ("q", "k", "v", "text_k", "text_v", "beta", "W_soft", "W_lin"):
+        assert np.array_equal(O._to_np(a[k]), O._to_np(b[k])), k
+    g = O._to_np(b["gates"])
+    assert g.shape == (2, cfg.B, cfg.L, cfg.H, cfg.d)
+    assert 0 < g.min() and g.max() < 1 and abs(g.mean() - 0.5) < 0.05

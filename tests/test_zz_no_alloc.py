@@ -13,32 +13,80 @@ import pytest
 import torch
 
 import softmax_attention_video_chunk_b200 as vdn
+from oracle import vdn_oracle as O
 from synth import CONFIGS, make_inputs
 from tests._parity import rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name,over,tol", [
-    ("tiny_f32", {}, 1e-5),
-    ("small_bf16", dict(T=16, N=96, H=4), 1e-4),
-    ("d128_bf16", dict(T=12, N=136, H=2, d=128), 1e-4),
+def _states(d, cfg, noalloc, **kw):
+    fn = vdn.vda_boundary_states_noalloc if noalloc else vdn.vda_boundary_states
+    return fn(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T, alpha=d["alpha"],
+              chunk=cfg.chunk, **kw)
+
+
+def _fill_scratch_with_another_problem():
+    """A larger problem (17 MiB of the 32 MiB array) first, so that the array
+    holds a different problem's contents when the checked calls start."""
+    cfg = CONFIGS["small_bf16"].replace(H=8, T=40, N=48, seed=23)
+    d = to_dev(make_inputs(cfg))
+    _states(d, cfg, True)
+    assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_OK"
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_f32", {}),
+    ("small_bf16", dict(T=16, N=96, H=4)),
+    ("d128_bf16", dict(T=12, N=136, H=2, d=128)),
+    ("d64_bf16_beta_per_token", dict(T=11, N=40, H=3)),
 ])
-def test_noalloc_matches_workspace_entry_twice(cuda_ok, name, over, tol):
+def test_noalloc_equals_workspace_entry_twice(cuda_ok, name, over):
+    """Same kernels, same inputs: the no-allocation call equals the workspace
+    call bit for bit, on two calls in a row, after a different problem has
+    left its contents in the static array; the status word reads VDN_OK."""
     base = CONFIGS["tiny_f32"] if name == "tiny_f32" else CONFIGS["small_bf16"].replace(seed=11)
     cfg = base.replace(**over)
+    tok = "beta_per_token" in name
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0), beta_per_token=tok)
+    d = to_dev(inp)
+    F_ref, G_ref = _states(d, cfg, False, beta_per_token=tok)
+    torch.cuda.synchronize()
+    _fill_scratch_with_another_problem()
+    for _ in range(2):  # the static scratch keeps the previous call's contents
+        F, G = _states(d, cfg, True, beta_per_token=tok)
+        assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_OK"
+        assert torch.equal(F, F_ref)
+        assert torch.equal(G, G_ref)
+
+
+def test_noalloc_matches_the_oracle(cuda_ok):
+    """The boundary states of the no-allocation call against the oracle's
+    literal frame-by-frame recurrence (tensor-core path, d = 128)."""
+    cfg = CONFIGS["small_bf16"].replace(T=12, N=136, H=2, d=128, seed=17)
     inp = make_inputs(cfg, alpha_range=(0.9, 1.0))
     d = to_dev(inp)
-    F_ref, G_ref = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                                           cfg.T, alpha=d["alpha"], chunk=cfg.chunk)
-    torch.cuda.synchronize()
-    for _ in range(2):  # the static scratch keeps the previous call's contents
-        F, G = vdn.vda_boundary_states_noalloc(d["k"], d["v"], d["beta"], d["text_k"],
-                                               d["text_v"], cfg.T, alpha=d["alpha"],
-                                               chunk=cfg.chunk)
-        torch.cuda.synchronize()
-        assert rel_err(F.double().cpu(), F_ref.double().cpu()) <= tol
-        assert rel_err(G.double().cpu(), G_ref.double().cpu()) <= tol
+    F, G = _states(d, cfg, True)
+    assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_OK"
+    Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+                               cfg.T, cfg.N, cfg.chunk, alpha=inp["alpha"])
+    assert rel_err(F.double().cpu(), Fo) <= 1e-4
+    assert rel_err(G.double().cpu(), Go) <= 1e-4
+
+
+def test_noalloc_reports_device_range_errors(cuda_ok):
+    """A value outside the fp16 range of the per-token statistics operand
+    sets VDN_ERR_RANGE in the array's status word, which the status reader
+    returns and clears; the next in-range call reads VDN_OK."""
+    cfg = CONFIGS["small_bf16"].replace(T=8, N=40, H=2, seed=5)
+    d = to_dev(make_inputs(cfg, beta_per_token=True))
+    bad = dict(d)
+    bad["v"] = d["v"] * 0 + 1e5  # representable in bf16, not in fp16
+    _states(bad, cfg, True, beta_per_token=True)
+    assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_ERR_RANGE"
+    assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_OK"  # read and cleared
+    _states(d, cfg, True, beta_per_token=True)
+    assert vdn.STATUS[vdn.noalloc_device_status()] == "VDN_OK"
 
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch(cuda_ok):
