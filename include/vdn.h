@@ -200,6 +200,60 @@ VDN_API vdn_status vdn_hybrid_attn_fwd_split(const vdn_params *p, const void *q,
                                      size_t workspace_bytes, vdn_stream_t stream,
                                      const vdn_stage_events *ev);
 
+/* ---- End to end from host memory ------------------------------------------
+ * One forward whose inputs and output live in host memory: the call enqueues
+ * the host -> device copies of every input, the forward, and the device ->
+ * host copy of `out`, ordered by CUDA events, on three caller streams.  It
+ * allocates no device memory: the device buffers of one step (a "slot") and
+ * the workspace are the caller's.  Alternating two slots lets the uploads of
+ * step i+1 and the download of step i-1 overlap the forward of step i; the
+ * events in the slot keep a slot's buffers from being overwritten while a
+ * previous step still reads them. */
+typedef struct vdn_host_inputs {
+  /* host pointers, same layouts and dtypes as vdn_hybrid_attn_fwd; pinned
+   * (page-locked) memory for asynchronous copies.  alpha may be NULL, and
+   * text_k / text_v when n_text == 0. */
+  const void *q, *k, *v;
+  const float *beta, *alpha;
+  const void *text_k, *text_v, *W_o_soft, *W_o_lin, *gates;
+} vdn_host_inputs;
+
+typedef struct vdn_host_slot {
+  /* device buffers of one step (caller-owned, sizes of the layouts above);
+   * alpha NULL when the host alpha is NULL */
+  void *q, *k, *v;
+  float *beta, *alpha;
+  void *text_k, *text_v, *W_o_soft, *W_o_lin, *gates, *out;
+  /* library-managed: zero-initialise the struct before its first use and
+   * release it with vdn_host_slot_release; three cudaEvent_t handles
+   * (uploaded, inputs read by the forward, output copied back) created on the
+   * slot's first use */
+  void *events[3];
+  int used;
+} vdn_host_slot;
+
+/* host_in: host inputs of this step; host_out: host memory for out
+ * [B, L, D_out] (out_dtype); slot: device buffers for this step; workspace as
+ * vdn_hybrid_attn_fwd.  copy_in / compute / copy_out: streams of the uploads,
+ * the forward and the download (they may all be the same stream).  On return
+ * *h2d_bytes and *d2h_bytes (each may be NULL) hold the bytes copied each way.
+ * Asynchronous: host_out is complete once copy_out reaches this point (for
+ * instance after cudaStreamSynchronize(copy_out)); host_in and the slot must
+ * stay untouched until then.  No source in the paper: the pages' serving stack
+ * moves data between host and GPU, and this is the library's form of it.
+ * Validation as vdn_hybrid_attn_fwd, plus every host and slot pointer the
+ * layouts require (VDN_ERR_INVALID_ARG). */
+VDN_API vdn_status vdn_hybrid_attn_fwd_host(const vdn_params *p, const vdn_host_inputs *host_in,
+                                            void *host_out, vdn_host_slot *slot,
+                                            void *workspace, size_t workspace_bytes,
+                                            vdn_stream_t copy_in, vdn_stream_t compute,
+                                            vdn_stream_t copy_out, size_t *h2d_bytes,
+                                            size_t *d2h_bytes);
+
+/* Destroys the events of a slot (after its last step has completed); the
+ * caller frees the slot's device buffers.  NULL is a no-op. */
+VDN_API vdn_status vdn_host_slot_release(vdn_host_slot *slot);
+
 /* ---- VDA-Prep: the linear branch's feature map ----------------------------
  * "Video DeltaNet" method (the linear branch applies its own feature map to
  * the pretrained projections: a separable short convolution of K and V -- a

@@ -109,6 +109,12 @@ def lib() -> ctypes.CDLL:
         L.vdn_text_query_attn.argtypes = [PP] + [_P] * 7 + [ctypes.c_size_t, _P]
         L.vdn_selftest_bounded_wait.restype = ctypes.c_int
         L.vdn_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint, _P]
+        L.vdn_hybrid_attn_fwd_host.restype = ctypes.c_int
+        L.vdn_hybrid_attn_fwd_host.argtypes = ([PP, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P,
+                                                ctypes.POINTER(ctypes.c_size_t),
+                                                ctypes.POINTER(ctypes.c_size_t)])
+        L.vdn_host_slot_release.restype = ctypes.c_int
+        L.vdn_host_slot_release.argtypes = [_P]
         L.vdn_selftest_exp2.restype = ctypes.c_int
         L.vdn_selftest_exp2.argtypes = [_P, _P, ctypes.c_size_t, _P]
         _lib = L
@@ -280,34 +286,105 @@ def vda_prep(q, k, v, wk_s, wk_t, wv_s, wv_t, T, grid_h, grid_w, *, l2_eps=1e-6,
 
 
 INPUT_NAMES = ("q", "k", "v", "beta", "alpha", "text_k", "text_v", "W_soft", "W_lin", "gates")
+_HOST_FIELDS = ("q", "k", "v", "beta", "alpha", "text_k", "text_v", "W_o_soft", "W_o_lin",
+                "gates")
 
 
-def hybrid_attn_fwd_host(host: dict, T, *, device_bufs=None, out_host=None, workspace=None,
+class VdnHostInputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _HOST_FIELDS]
+
+
+class VdnHostSlot(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_void_p) for n in _HOST_FIELDS] + [("out", ctypes.c_void_p)] +
+                [("events", ctypes.c_void_p * 3), ("used", ctypes.c_int)])
+
+
+def _host_ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("host tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+class HostSlot:
+    """Device buffers of one end-to-end step (vdn_host_slot): inputs shaped
+    like ``host_example`` and ``out``; the slot's events are released with
+    the object (after the device is done with them)."""
+
+    def __init__(self, host_example: dict, p: VdnParams, device):
+        import torch
+        self.bufs = {n: (None if host_example.get(n) is None else
+                         torch.empty_like(host_example[n], device=device)) for n in INPUT_NAMES}
+        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
+        self.out = torch.empty(p.B, p.T * p.N, p.D_out, dtype=odt, device=device)
+        self.c = VdnHostSlot()
+        for f, n in zip(_HOST_FIELDS, INPUT_NAMES):
+            setattr(self.c, f, _ptr(self.bufs[n]))
+        self.c.out = _ptr(self.out)
+
+    def release(self):
+        if self.c is not None:
+            lib().vdn_host_slot_release(ctypes.byref(self.c))
+            self.c = None
+
+    def __del__(self):
+        try:
+            self.release()
+        except Exception:
+            pass
+
+
+def _host_inputs(host: dict) -> VdnHostInputs:
+    hi = VdnHostInputs()
+    for f, n in zip(_HOST_FIELDS, INPUT_NAMES):
+        setattr(hi, f, _host_ptr(host.get(n)))
+    return hi
+
+
+def host_fwd_step(p: VdnParams, host: dict, out_host, slot: HostSlot, workspace, s_in, s_cmp,
+                  s_out):
+    """One end-to-end step through vdn_hybrid_attn_fwd_host: uploads on
+    ``s_in``, the forward on ``s_cmp``, the download into ``out_host`` on
+    ``s_out`` (torch streams).  Returns (h2d_bytes, d2h_bytes)."""
+    h2d, d2h = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    hi = _host_inputs(host)
+    rc = lib().vdn_hybrid_attn_fwd_host(ctypes.byref(p), ctypes.byref(hi), _host_ptr(out_host),
+                                        ctypes.byref(slot.c), _ptr(workspace), workspace.numel(),
+                                        _stream(s_in), _stream(s_cmp), _stream(s_out),
+                                        ctypes.byref(h2d), ctypes.byref(d2h))
+    if rc != 0:
+        raise VdnError(rc, "vdn_hybrid_attn_fwd_host")
+    return h2d.value, d2h.value
+
+
+def hybrid_attn_fwd_host(host: dict, T, *, slot=None, out_host=None, workspace=None,
                          stream=None, params=None, **kw):
-    """End-to-end call on host (pinned) tensors: copies every input to the
-    device, runs the forward, and copies ``out`` back into ``out_host``, all on
-    one stream.  ``device_bufs`` (same keys) are reused device buffers.
-    Returns (out_host, h2d_bytes, d2h_bytes)."""
+    """End-to-end call on host (pinned) tensors through vdn_hybrid_attn_fwd_host:
+    every input copied to the device, the forward, and ``out`` copied back into
+    ``out_host``, all on one stream.  ``slot`` (a HostSlot) holds reusable
+    device buffers.  Returns (out_host, h2d_bytes, d2h_bytes); out_host is
+    complete after the stream synchronises."""
     import torch
     dev = torch.device("cuda", torch.cuda.current_device())
     s = torch.cuda.current_stream() if stream is None else stream
-    with torch.cuda.stream(s):
-        if device_bufs is None:
-            device_bufs = {n: (None if host.get(n) is None else
-                               torch.empty_like(host[n], device=dev)) for n in INPUT_NAMES}
-        h2d = 0
-        for n in INPUT_NAMES:
-            if host.get(n) is not None:
-                device_bufs[n].copy_(host[n], non_blocking=True)
-                h2d += host[n].numel() * host[n].element_size()
-        d = device_bufs
-        out = hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                              d["W_soft"], d["W_lin"], d["gates"], T, alpha=d.get("alpha"),
-                              workspace=workspace, stream=s, params=params, **kw)
-        if out_host is None:
-            out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        out_host.copy_(out, non_blocking=True)
-    return out_host, h2d, out.numel() * out.element_size()
+    if params is None:
+        W = host["W_soft"]
+        D_out = W.shape[1]
+        B, L, H, d = host["q"].shape
+        n_text = 0 if host.get("text_k") is None else host["text_k"].shape[1]
+        params = make_params(B, H, T, L // T, d, n_text, _dtype_name(host["q"]), D_out=D_out,
+                             **kw)
+    p = params
+    slot = HostSlot(host, p, dev) if slot is None else slot
+    ws = alloc_workspace(p, dev) if workspace is None else workspace
+    if out_host is None:
+        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
+        out_host = torch.empty(p.B, p.T * p.N, p.D_out, dtype=odt, pin_memory=True)
+    h2d, d2h = host_fwd_step(p, host, out_host, slot, ws, s, s, s)
+    return out_host, h2d, d2h
 
 
 def hybrid_attn_branches(q, k, v, beta, text_k, text_v, T, *, alpha=None, workspace=None,
@@ -406,12 +483,13 @@ def use_tc_params(p: VdnParams) -> bool:
 class HostPipeline:
     """End-to-end forwards on host (pinned) tensors with the copies overlapped.
 
-    Each ``submit`` enqueues: host -> device copies of every input (copy
-    stream), the forward (compute stream), and the device -> host copy of
-    ``out`` (copy-back stream), ordered by CUDA events.  Two slots of device
-    buffers alternate, so step i+1's uploads and step i-1's download run while
-    step i computes.  Host input and output tensors must stay untouched until
-    ``synchronize`` (or until the slot is reused two steps later).
+    Each ``submit`` is one vdn_hybrid_attn_fwd_host call: host -> device copies
+    of every input (copy stream), the forward (compute stream), and the
+    device -> host copy of ``out`` (copy-back stream), ordered by the events of
+    the step's slot.  Two slots of device buffers alternate, so step i+1's
+    uploads and step i-1's download run while step i computes.  Host input and
+    output tensors must stay untouched until ``synchronize`` (or until the slot
+    is reused two steps later).
     """
 
     def __init__(self, host_example: dict, T, *, params=None, **kw):
@@ -419,19 +497,14 @@ class HostPipeline:
         self.T = T
         dev = torch.device("cuda", torch.cuda.current_device())
         self.dev = dev
-        d0 = {n: (None if host_example.get(n) is None else
-                  torch.empty_like(host_example[n], device=dev)) for n in INPUT_NAMES}
-        self.params = params or params_for(d0["q"], d0["v"], d0["text_k"], T, d0["W_soft"], **kw)
-        p = self.params
-        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
-        self.slots = []
-        for s in range(2):
-            bufs = d0 if s == 0 else {n: (None if v is None else torch.empty_like(v))
-                                      for n, v in d0.items()}
-            out = torch.empty(p.B, p.T * p.N, p.D_out, dtype=odt, device=dev)
-            self.slots.append({"in": bufs, "out": out,
-                               "inputs_free": torch.cuda.Event(), "out_free": torch.cuda.Event(),
-                               "used": False})
+        if params is None:
+            q, W = host_example["q"], host_example["W_soft"]
+            B, L, H, d = q.shape
+            tk = host_example.get("text_k")
+            params = make_params(B, H, T, L // T, d, 0 if tk is None else tk.shape[1],
+                                 _dtype_name(q), D_out=W.shape[1], **kw)
+        self.params = p = params
+        self.slots = [HostSlot(host_example, p, dev) for _ in range(2)]
         self.ws = alloc_workspace(p, dev)
         self.s_h2d = torch.cuda.Stream(dev)
         self.s_cmp = torch.cuda.Stream(dev)
@@ -440,37 +513,21 @@ class HostPipeline:
 
     def submit(self, host: dict, out_host):
         """Enqueue one forward; returns (h2d_bytes, d2h_bytes)."""
-        import torch
         slot = self.slots[self.step % 2]
         self.step += 1
-        up, done = torch.cuda.Event(), torch.cuda.Event()
-        h2d = 0
-        with torch.cuda.stream(self.s_h2d):
-            if slot["used"]:
-                self.s_h2d.wait_event(slot["inputs_free"])
-            for n in INPUT_NAMES:
-                if host.get(n) is not None:
-                    slot["in"][n].copy_(host[n], non_blocking=True)
-                    h2d += host[n].numel() * host[n].element_size()
-            up.record(self.s_h2d)
-        with torch.cuda.stream(self.s_cmp):
-            self.s_cmp.wait_event(up)
-            if slot["used"]:
-                self.s_cmp.wait_event(slot["out_free"])
-            d = slot["in"]
-            hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                            d["W_soft"], d["W_lin"], d["gates"], self.T, alpha=d.get("alpha"),
-                            out=slot["out"], workspace=self.ws, stream=self.s_cmp,
-                            params=self.params)
-            slot["inputs_free"].record(self.s_cmp)
-            done.record(self.s_cmp)
-        with torch.cuda.stream(self.s_d2h):
-            self.s_d2h.wait_event(done)
-            out_host.copy_(slot["out"], non_blocking=True)
-            slot["out_free"].record(self.s_d2h)
-        slot["used"] = True
-        return h2d, slot["out"].numel() * slot["out"].element_size()
+        return host_fwd_step(self.params, host, out_host, slot, self.ws, self.s_h2d, self.s_cmp,
+                             self.s_d2h)
+
+    def inputs_read_event(self, i: int):
+        """cudaEvent_t handle (int) recorded after the forward of slot i read
+        its inputs (valid once the slot was used)."""
+        return self.slots[i].c.events[1]
 
     def synchronize(self):
         for s in (self.s_h2d, self.s_cmp, self.s_d2h):
             s.synchronize()
+
+    def close(self):
+        self.synchronize()
+        for sl in self.slots:
+            sl.release()

@@ -39,6 +39,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase (never suspends the thread): several of these
+// can be in flight at once, unlike a chain of blocking waits.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -284,6 +297,41 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;             // 128-byte swizzle
   return d;
+}
+
+// The same descriptor split into its two 32-bit words: the low word holds the
+// start address (>> 4) and the leading byte offset, the high word the stride
+// byte offset, version and swizzle mode, which are the same for every K-major
+// 128-byte-swizzled operand.  Moving the start address by `off` bytes (a
+// multiple of 16 inside shared memory) adds off >> 4 to the low word, so an
+// MMA issue loop can step through K with one 32-bit add per operand.
+__device__ __forceinline__ uint32_t sdesc_k_sw128_lo(uint32_t saddr) {
+  return ((saddr & 0x3FFFFu) >> 4) | (1u << 16);
+}
+constexpr uint32_t kSdescKSw128Hi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+// D[tmem] (+)= A[smem] * B[smem]^T from the low descriptor words.
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %5};\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescKSw128Hi)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T from the low descriptor word of B.
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescKSw128Hi)
+      : "memory");
 }
 
 // Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle: rows of

@@ -405,6 +405,92 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_params* p, const void* q, const void* k
                                     gates, out, workspace, workspace_bytes, stream, nullptr);
 }
 
+vdn_status vdn_hybrid_attn_fwd_host(const vdn_params* p, const vdn_host_inputs* hin,
+                                    void* host_out, vdn_host_slot* slot, void* workspace,
+                                    size_t workspace_bytes, vdn_stream_t copy_in,
+                                    vdn_stream_t compute, vdn_stream_t copy_out,
+                                    size_t* h2d_bytes, size_t* d2h_bytes) {
+  VDN_TRY(validate_params(p));
+  if (hin == nullptr || slot == nullptr || host_out == nullptr) return VDN_ERR_INVALID_ARG;
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  const size_t es = p->dtype == VDN_BF16 ? 2 : 4;
+  const size_t B = p->B, H = p->H, L = (size_t)p->T * p->N, d = p->d_k, nt = p->n_text;
+  const size_t act = B * L * H * d * es;
+  const size_t beta_n = (p->flags & VDN_FLAG_BETA_PER_TOKEN) ? B * H * (nt + L)
+                                                              : B * H * (p->T + 1);
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t bytes;
+    bool required;
+  };
+  const Copy cp[10] = {
+      {slot->q, hin->q, act, true},
+      {slot->k, hin->k, act, true},
+      {slot->v, hin->v, act, true},
+      {slot->beta, hin->beta, beta_n * 4, true},
+      {slot->alpha, hin->alpha, B * H * p->T * d * 4, false},
+      {slot->text_k, hin->text_k, B * nt * H * d * es, nt > 0},
+      {slot->text_v, hin->text_v, B * nt * H * d * es, nt > 0},
+      {slot->W_o_soft, hin->W_o_soft, H * d * (size_t)p->D_out * es, true},
+      {slot->W_o_lin, hin->W_o_lin, H * d * (size_t)p->D_out * es, true},
+      {slot->gates, hin->gates, 2 * act, true},
+  };
+  for (const Copy& c : cp) {
+    if (c.required && (c.src == nullptr || c.dst == nullptr)) return VDN_ERR_INVALID_ARG;
+    if ((c.src == nullptr) != (c.dst == nullptr)) return VDN_ERR_INVALID_ARG;
+    VDN_TRY(check_ptr(c.dst, false));
+  }
+  VDN_TRY(check_ptr(slot->out, true));
+  const size_t out_bytes = B * L * (size_t)p->D_out * (p->out_dtype == VDN_BF16 ? 2 : 4);
+  cudaStream_t s_in = (cudaStream_t)copy_in, s_cmp = (cudaStream_t)compute,
+               s_out = (cudaStream_t)copy_out;
+  cudaEvent_t* ev = reinterpret_cast<cudaEvent_t*>(slot->events);
+  if (!slot->used)
+    for (int i = 0; i < 3; ++i) {
+      if (ev[i] == nullptr &&
+          cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess)
+        return VDN_ERR_CUDA;
+    }
+  cudaEvent_t uploaded = ev[0], inputs_read = ev[1], out_copied = ev[2];
+  // uploads: once the previous forward on this slot has read its inputs
+  if (slot->used) VDN_CUDA(cudaStreamWaitEvent(s_in, inputs_read, 0));
+  size_t h2d = 0;
+  for (const Copy& c : cp) {
+    if (c.src == nullptr) continue;
+    VDN_CUDA(cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s_in));
+    h2d += c.bytes;
+  }
+  VDN_CUDA(cudaEventRecord(uploaded, s_in));
+  // forward: once uploaded and the previous download of this slot's out is done
+  VDN_CUDA(cudaStreamWaitEvent(s_cmp, uploaded, 0));
+  if (slot->used) VDN_CUDA(cudaStreamWaitEvent(s_cmp, out_copied, 0));
+  VDN_TRY(fwd_impl(p, slot->q, slot->k, slot->v, slot->q, slot->k, slot->v, slot->beta,
+                   slot->alpha, slot->text_k, slot->text_v, slot->W_o_soft, slot->W_o_lin,
+                   slot->gates, slot->out, workspace, workspace_bytes, compute, nullptr));
+  VDN_CUDA(cudaEventRecord(inputs_read, s_cmp));
+  // download
+  VDN_CUDA(cudaStreamWaitEvent(s_out, inputs_read, 0));
+  VDN_CUDA(cudaMemcpyAsync(host_out, slot->out, out_bytes, cudaMemcpyDeviceToHost, s_out));
+  VDN_CUDA(cudaEventRecord(out_copied, s_out));
+  slot->used = 1;
+  if (h2d_bytes != nullptr) *h2d_bytes = h2d;
+  if (d2h_bytes != nullptr) *d2h_bytes = out_bytes;
+  return VDN_OK;
+}
+
+vdn_status vdn_host_slot_release(vdn_host_slot* slot) {
+  if (slot == nullptr) return VDN_OK;
+  cudaEvent_t* ev = reinterpret_cast<cudaEvent_t*>(slot->events);
+  vdn_status st = VDN_OK;
+  for (int i = 0; i < 3; ++i) {
+    if (ev[i] != nullptr && cudaEventDestroy(ev[i]) != cudaSuccess) st = VDN_ERR_CUDA;
+    ev[i] = nullptr;
+  }
+  slot->used = 0;
+  return st;
+}
+
 vdn_status vdn_prep_params_init(vdn_prep_params* p, int B, int H, int T, int grid_h,
                                 int grid_w, int d, vdn_dtype dtype) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;

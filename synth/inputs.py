@@ -82,6 +82,10 @@ CONFIGS = {
     # on the device in total)
     "768p_h4_bf16": Config("768p_h4_bf16", B=1, H=4, T=75, N=1536, d=128, n_text=512,
                            dtype="bf16", seed=2, q_norm=True),
+    # the batched clips with 4 of their 16 batch items: the profiler workload
+    # of the VDA state kernels (inputs > L2, about 1.5 GB on the device)
+    "batched_b4_bf16": Config("batched_b4_bf16", B=4, H=16, T=20, N=576, d=128,
+                              n_text=256, dtype="bf16", seed=4, q_norm=True),
 }
 
 _TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -201,3 +201,44 @@ def test_frozen_state_flag_is_accepted():
     p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", frozen_state=True)
     assert p.flags & vdn.FLAG_FROZEN_STATE
     assert vdn.workspace_bytes(p) == vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8))
+
+
+def test_host_entry_validates_before_any_copy():
+    """vdn_hybrid_attn_fwd_host checks the host inputs, the slot's device
+    buffers and the workspace before it enqueues anything."""
+    L = vdn.lib()
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    need = vdn.workspace_bytes(p)
+    ws = 0x7f0000000000
+    hi = vdn.VdnHostInputs()
+    slot = vdn.VdnHostSlot()
+    for i, f in enumerate(vdn._HOST_FIELDS):
+        setattr(hi, f, 0x100000 + 0x1000 * i)
+        setattr(slot, f, 0x200000 + 0x1000 * i)
+    hi.alpha = slot.alpha = None
+    slot.out = 0x300000
+
+    def call(host_in=hi, out=0x400000, sl=slot, w=ws, nbytes=need):
+        h2d, d2h = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        return vdn.STATUS[L.vdn_hybrid_attn_fwd_host(
+            ctypes.byref(p), None if host_in is None else ctypes.byref(host_in), out,
+            None if sl is None else ctypes.byref(sl), w, nbytes, None, None, None,
+            ctypes.byref(h2d), ctypes.byref(d2h))]
+
+    assert call(host_in=None) == "VDN_ERR_INVALID_ARG"
+    assert call(sl=None) == "VDN_ERR_INVALID_ARG"
+    assert call(out=None) == "VDN_ERR_INVALID_ARG"
+    assert call(nbytes=need - 1) == "VDN_ERR_WORKSPACE"
+    assert call(w=ws + 64) == "VDN_ERR_ALIGNMENT"
+    hi.alpha = 0x500000  # a host alpha without a device buffer for it
+    assert call() == "VDN_ERR_INVALID_ARG"
+    hi.alpha = None
+    slot.gates = None  # a required device buffer missing
+    assert call() == "VDN_ERR_INVALID_ARG"
+    slot.gates = 0x200008  # misaligned
+    assert call() == "VDN_ERR_ALIGNMENT"
+    slot.gates = 0x209000
+    slot.out = None
+    assert call() == "VDN_ERR_INVALID_ARG"
+    assert slot.used == 0 and all(e is None for e in slot.events)  # nothing was created
+    assert L.vdn_host_slot_release(None) == 0
