@@ -114,6 +114,15 @@ typedef struct CUstream_st *vdn_stream_t;
  * likewise, S_text = W_text).  Keys are taken as given: SANA-WM's frame-size
  * key scaling, whose factor the pages lost, is left to the caller. */
 #define VDN_FLAG_FROZEN_STATE (1u << 4)
+/* How the bidirectional scan (implementation section, "Chunk-wise scans") is
+ * evaluated.  By default the library picks, from the problem's shape, either
+ * the composition of each chunk's frame maps followed by a scan over chunks,
+ * or a scan straight over the frames that keeps only the chunk-boundary
+ * states (fewer products, more sequential steps: the better choice for short
+ * clips).  Both give the same states up to FP32 rounding.  These flags force
+ * one of them (setting both is VDN_ERR_INVALID_ARG). */
+#define VDN_FLAG_SCAN_FRAMES (1u << 5)
+#define VDN_FLAG_SCAN_CHUNKS (1u << 6)
 
 typedef struct vdn_params {
   int B;             /* batch */

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libvdn.so")
 VDN_F32, VDN_BF16 = 0, 1
 FLAG_TEXT_FULL, FLAG_SIMT, FLAG_TEXT_SOFTMAX, FLAG_BETA_PER_TOKEN = 1, 2, 4, 8
 FLAG_FROZEN_STATE = 16
+FLAG_SCAN_FRAMES, FLAG_SCAN_CHUNKS = 32, 64
 
 STATUS = {
     0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_SHAPE", 3: "VDN_ERR_DTYPE",
@@ -124,7 +125,7 @@ def lib() -> ctypes.CDLL:
 def make_params(B, H, T, N, d, n_text, dtype="bf16", *, chunk=5, window_radius=1,
                 D_out=None, out_dtype="f32", softmax_scale=0.0, rms_eps=1e-6,
                 text_full=False, simt=False, text_softmax=False,
-                beta_per_token=False, frozen_state=False) -> VdnParams:
+                beta_per_token=False, frozen_state=False, scan=None) -> VdnParams:
     p = VdnParams()
     dt = {"f32": VDN_F32, "bf16": VDN_BF16}
     rc = lib().vdn_params_init(ctypes.byref(p), B, H, T, N, d, n_text, dt[dtype])
@@ -135,7 +136,8 @@ def make_params(B, H, T, N, d, n_text, dtype="bf16", *, chunk=5, window_radius=1
     p.flags = ((FLAG_TEXT_FULL if text_full else 0) | (FLAG_SIMT if simt else 0) |
                (FLAG_TEXT_SOFTMAX if text_softmax else 0) |
                (FLAG_BETA_PER_TOKEN if beta_per_token else 0) |
-               (FLAG_FROZEN_STATE if frozen_state else 0))
+               (FLAG_FROZEN_STATE if frozen_state else 0) |
+               {None: 0, "frames": FLAG_SCAN_FRAMES, "chunks": FLAG_SCAN_CHUNKS}[scan])
     size = ctypes.c_size_t(0)
     rc = lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
     if rc != 0:

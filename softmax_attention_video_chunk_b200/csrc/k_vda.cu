@@ -26,6 +26,7 @@
 #include "vdn_kernels.h"
 
 namespace vdn {
+int sm_count();
 
 // ---------------------------------------------------------------------------
 // S1 + S2: frame statistics and Gauss-Jordan solve
@@ -342,6 +343,129 @@ vda_chunk_scan_kernel(const float* __restrict__ Rf, const float* __restrict__ CM
 }
 
 // ---------------------------------------------------------------------------
+// S3+S4 for short clips: the bidirectional scan run directly over the frames,
+// S <- M_t S + R_t, keeping only the chunk-boundary states (FS[k] after the
+// frames of chunks < k, GS[k] after the frames of chunks >= k).  It needs T
+// sequential steps instead of ceil(T / C), but does one product per frame
+// instead of the composition's two per frame plus the chunk scan, and reads
+// the per-frame maps directly.  Anchor frames (no write) only decay:
+// S <- Diag(alpha_t) S.  One CTA per 32-column slice of S and direction.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf,
+                      const float* __restrict__ alpha, float* __restrict__ FS,
+                      float* __restrict__ GS, int B, int H, int T, int C, float init_scale) {
+  constexpr int RT = D / 32, SD = D + 4;  // row stride keeps float4 stores aligned
+  const int cb = blockIdx.x * 32, h = blockIdx.y, b = blockIdx.z >> 1, dir = blockIdx.z & 1;
+  const int nc = (T + C - 1) / C;
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+  const size_t mat = (size_t)D * D;
+  const size_t bh = (size_t)b * H + h;
+  extern __shared__ float smem[];
+  float* Ms = smem;          // [D][SD]
+  float* Ss = Ms + D * SD;   // [D][32]
+  const float* St = Rf + (bh * (T + 1) + 0) * mat;  // text state
+  for (int q = tid; q < D * 32; q += blockDim.x) {
+    const int i = q >> 5, j = q & 31;
+    Ss[q] = init_scale * St[i * D + cb + j];
+  }
+  float* OUT = dir == 0 ? FS : GS;
+  __syncthreads();
+  {
+    const int k0 = dir == 0 ? 0 : nc;
+    for (int q = tid; q < D * 32; q += blockDim.x) {
+      const int i = q >> 5, j = q & 31;
+      OUT[(bh * (nc + 1) + k0) * mat + i * D + cb + j] = Ss[q];
+    }
+  }
+  // M_t of the next frame is loaded into registers (D*D/4/256 float4 per
+  // thread, all in flight at once) while the current frame's product runs
+  constexpr int NV = D * D / 4 / 256;
+  float4 mv[NV];
+  auto frame_of = [&](int step) { return dir == 0 ? step : T - 1 - step; };
+  auto is_anchor = [&](int t) { return t == 0 || t == T - 1; };
+  auto load_m = [&](int t) {
+    const float4* Mg = reinterpret_cast<const float4*>(Mf + (bh * (T + 1) + 1 + t) * mat);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) mv[k] = Mg[tid + k * 256];
+  };
+  if (T > 0 && !is_anchor(frame_of(0))) load_m(frame_of(0));
+  for (int step = 0; step < T; ++step) {
+    const int t = frame_of(step);
+    const bool anchor = is_anchor(t);
+    const float* Rg = Rf + (bh * (T + 1) + 1 + t) * mat;
+    float acc[RT][4];
+    __syncthreads();
+    if (anchor) {  // M_t = Diag(alpha_t), R_t = 0
+      const float* al = alpha != nullptr ? alpha + (bh * T + t) * D : nullptr;
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const int i = ty * RT + r;
+        const float a = al != nullptr ? al[i] : 1.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[r][m] = a * Ss[i * 32 + tx * 4 + m];
+      }
+      if (step + 1 < T && !is_anchor(frame_of(step + 1))) load_m(frame_of(step + 1));
+    } else {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int q = tid + k * 256;
+        const int i = q / (D / 4), c4 = q % (D / 4);
+        *reinterpret_cast<float4*>(Ms + i * SD + 4 * c4) = mv[k];
+      }
+      __syncthreads();
+      if (step + 1 < T && !is_anchor(frame_of(step + 1))) load_m(frame_of(step + 1));
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[r][m] = 0.f;
+#pragma unroll 4
+      for (int l = 0; l < D; ++l) {
+        const float4 sv = *reinterpret_cast<const float4*>(Ss + l * 32 + tx * 4);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float a = Ms[(ty * RT + r) * SD + l];
+          acc[r][0] = fmaf(a, sv.x, acc[r][0]);
+          acc[r][1] = fmaf(a, sv.y, acc[r][1]);
+          acc[r][2] = fmaf(a, sv.z, acc[r][2]);
+          acc[r][3] = fmaf(a, sv.w, acc[r][3]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const int i = ty * RT + r;
+        const float4 rv = *reinterpret_cast<const float4*>(Rg + i * D + cb + tx * 4);
+        acc[r][0] += rv.x;
+        acc[r][1] += rv.y;
+        acc[r][2] += rv.z;
+        acc[r][3] += rv.w;
+      }
+    }
+    __syncthreads();
+    // chunk boundary reached after this frame: forward after the last frame of
+    // chunk k-1 (k = (t+1)/C, or nc after the last frame), reverse after the
+    // first frame of chunk k = t/C
+    int kout = -1;
+    if (dir == 0) {
+      if (t == T - 1) kout = nc;
+      else if ((t + 1) % C == 0) kout = (t + 1) / C;
+    } else if (t % C == 0) {
+      kout = t / C;
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const int i = ty * RT + r;
+      *reinterpret_cast<float4*>(Ss + i * 32 + tx * 4) =
+          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      if (kout >= 0)
+        *reinterpret_cast<float4*>(OUT + (bh * (nc + 1) + kout) * mat + i * D + cb + tx * 4) =
+            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // S6: readout with the decay bridge, per frame (CUDA cores, FP32).
 // ---------------------------------------------------------------------------
 template <int D, typename TIn>
@@ -440,6 +564,27 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
         (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.text_k, (const TIn*)a.text_v, a.beta,
         a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text, a.beta_tok, a.frozen);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // Chunk composition + chunk scan, or the direct frame scan: whichever the
+  // wave-count model puts first.  Sequential steps per CTA: composition
+  // 2 (C - 1) products then nc scan steps; direct scan T products.  CTAs: the
+  // composition runs 2 B H nc (D / 32) of them, both scans 2 B H (D / 32);
+  // two CTAs per SM.
+  const long long slots = 2LL * sm_count();
+  const long long cta_scan = 2LL * B * H * (D / 32);
+  const long long cta_comp = cta_scan * nc;
+  const long long waves_scan = (cta_scan + slots - 1) / slots;
+  const long long waves_comp = (cta_comp + slots - 1) / slots;
+  const long long cost_chunk = waves_comp * 2LL * (a.C - 1) + waves_scan * nc;
+  const long long cost_direct = waves_scan * (long long)T;
+  if (a.scan_mode == 1 || (a.scan_mode == 0 && cost_direct <= cost_chunk)) {
+    const size_t sm = sizeof(float) * ((size_t)D * (D + 4) + (size_t)D * 32);
+    auto kern = vda_frame_scan_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(D / 32, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.alpha, a.FS, a.GS, B, H, T, a.C,
+                                                  a.init_scale);
+    return cudaGetLastError();
   }
   {
     const size_t sm = sizeof(float) * ((size_t)D * (D + 1) + 2 * (size_t)D * 32);

@@ -55,7 +55,8 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   const int NS = beta_tok ? 2 : 3;
   const int SSTR = beta_tok ? 3 * STB : STB;  // stage stride
   constexpr int NN = 2 * D;               // MMA N (columns of D)
-  constexpr int SD = D + 1;               // padded row stride of the FP32 matrices
+  constexpr int SD = D + 1;               // padded row stride of I + beta A, then X
+  constexpr int SDW = D + 4;              // row stride of beta W (float4-aligned rows)
   constexpr int BL = D / 16;              // register block edge per thread
 
   const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -89,8 +90,8 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   // phase 1: TMA ring; phase 2 (after the MMAs): the two FP32 matrices
   uint8_t* stages = smem;
   float* Ash = (float*)smem;           // [D][SD]  I + beta A, then X
-  float* Wsh = Ash + D * SD;           // [D][SD]  beta W
-  constexpr int MATB = 2 * D * SD * 4;
+  float* Wsh = Ash + D * SD;           // [D][SDW] beta W
+  constexpr int MATB = (D * SD + D * SDW) * 4;
   constexpr int RING = 6 * STB;  // the larger of 3 x STB and 2 x 3 x STB
   constexpr int BIG = (RING > MATB) ? RING : MATB;
   uint64_t* full = (uint64_t*)(smem + ((BIG + 1023) & ~1023));
@@ -252,7 +253,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
           if (part == 0)  // I + beta A (VDA), or I - beta A (frozen-state rule)
             Ash[i * SD + j] = (frozen ? -x : x) + (i == j ? 1.f : 0.f);
           else
-            Wsh[i * SD + j] = x;
+            Wsh[i * SDW + j] = x;
         }
       }
     }
@@ -325,7 +326,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
     for (int i = 0; i < BL; ++i) {
       float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
-      const float* src = Wsh + (ty * BL + i) * SD + tx * BL;
+      const float* src = Wsh + (ty * BL + i) * SDW + tx * BL;
 #pragma unroll
       for (int c = 0; c < BL; c += 4)
         *reinterpret_cast<float4*>(dst + c) = make_float4(src[c], src[c + 1], src[c + 2], src[c + 3]);
@@ -338,6 +339,11 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
     for (int c = 0; c < BL; ++c) Ash[(ty * BL + i) * SD + tx * BL + c] = a[i][c];
   __syncthreads();
+  // R = X W: thread (ty, tx) computes rows ty*BL .. +BL-1 and the column
+  // groups {4 tx .. 4 tx + 3} + 4 D/4 g for g < BL/4 (groups of four columns,
+  // D/4 apart), so that the sixteen threads of a row group read W as
+  // consecutive float4 (no shared-memory bank conflicts)
+  constexpr int NGR = BL / 4;
   float acc[BL][BL];
 #pragma unroll
   for (int i = 0; i < BL; ++i)
@@ -349,7 +355,13 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
     for (int i = 0; i < BL; ++i) xv[i] = Ash[(ty * BL + i) * SD + l];
 #pragma unroll
-    for (int c = 0; c < BL; ++c) wv[c] = Wsh[l * SD + tx * BL + c];
+    for (int g = 0; g < NGR; ++g) {
+      const float4 w4 = *reinterpret_cast<const float4*>(Wsh + l * SDW + g * (D / NGR) + tx * 4);
+      wv[4 * g] = w4.x;
+      wv[4 * g + 1] = w4.y;
+      wv[4 * g + 2] = w4.z;
+      wv[4 * g + 3] = w4.w;
+    }
 #pragma unroll
     for (int i = 0; i < BL; ++i)
 #pragma unroll
@@ -357,11 +369,11 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   }
 #pragma unroll
   for (int i = 0; i < BL; ++i) {
-    float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
+    float* dst = Ro + (size_t)(ty * BL + i) * D + tx * 4;
 #pragma unroll
-    for (int c = 0; c < BL; c += 4)
-      *reinterpret_cast<float4*>(dst + c) =
-          make_float4(acc[i][c], acc[i][c + 1], acc[i][c + 2], acc[i][c + 3]);
+    for (int g = 0; g < NGR; ++g)
+      *reinterpret_cast<float4*>(dst + g * (D / NGR)) =
+          make_float4(acc[i][4 * g], acc[i][4 * g + 1], acc[i][4 * g + 2], acc[i][4 * g + 3]);
   }
 }
 

@@ -65,7 +65,10 @@ static WsLayout layout(const vdn_params& p) {
 static vdn_status validate_params(const vdn_params* p) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;
   if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT | VDN_FLAG_TEXT_SOFTMAX |
-                             VDN_FLAG_BETA_PER_TOKEN | VDN_FLAG_FROZEN_STATE))
+                             VDN_FLAG_BETA_PER_TOKEN | VDN_FLAG_FROZEN_STATE |
+                             VDN_FLAG_SCAN_FRAMES | VDN_FLAG_SCAN_CHUNKS))
+    return VDN_ERR_INVALID_ARG;
+  if ((p->flags & VDN_FLAG_SCAN_FRAMES) && (p->flags & VDN_FLAG_SCAN_CHUNKS))
     return VDN_ERR_INVALID_ARG;
   if ((p->dtype != VDN_F32 && p->dtype != VDN_BF16) ||
       (p->out_dtype != VDN_F32 && p->out_dtype != VDN_BF16))
@@ -151,6 +154,7 @@ static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const
   a.tc = use_tc(*p);
   a.beta_tok = (p->flags & VDN_FLAG_BETA_PER_TOKEN) != 0;
   a.frozen = (p->flags & VDN_FLAG_FROZEN_STATE) != 0;
+  a.scan_mode = (p->flags & VDN_FLAG_SCAN_FRAMES) ? 1 : ((p->flags & VDN_FLAG_SCAN_CHUNKS) ? 2 : 0);
   a.status = (int*)(ws + w.status);
   return a;
 }

@@ -19,6 +19,7 @@ struct VdaArgs {
   bool tc;      // frame statistics on the tensor cores (bf16, d in {64, 128})
   bool beta_tok;  // beta per token: [B][H][n_text + L]
   bool frozen;    // frozen-state rule: M = (I - A) Diag(alpha), R = W (no inverse)
+  int scan_mode;  // 0: chosen from the shape; 1: scan over frames; 2: compose chunks
   int* status;  // device status word
 };
 

@@ -53,7 +53,7 @@ def test_params_init_defaults():
     ("chunk", 0, "VDN_ERR_SHAPE"), ("window_radius", -1, "VDN_ERR_SHAPE"),
     ("n_text", -1, "VDN_ERR_SHAPE"), ("D_out", 12, "VDN_ERR_SHAPE"),
     ("d_v", 32, "VDN_ERR_UNSUPPORTED"), ("dtype", 7, "VDN_ERR_DTYPE"),
-    ("out_dtype", 3, "VDN_ERR_DTYPE"), ("flags", 1 << 5, "VDN_ERR_INVALID_ARG"),
+    ("out_dtype", 3, "VDN_ERR_DTYPE"), ("flags", 1 << 7, "VDN_ERR_INVALID_ARG"),
     ("softmax_scale", -1.0, "VDN_ERR_INVALID_ARG"), ("rms_eps", float("nan"), "VDN_ERR_INVALID_ARG"),
 ])
 def test_param_validation(field, value, code):
@@ -242,3 +242,14 @@ def test_host_entry_validates_before_any_copy():
     assert call() == "VDN_ERR_INVALID_ARG"
     assert slot.used == 0 and all(e is None for e in slot.events)  # nothing was created
     assert L.vdn_host_slot_release(None) == 0
+
+
+def test_scan_flags_are_exclusive():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    size = ctypes.c_size_t(0)
+    for f in (vdn.FLAG_SCAN_FRAMES, vdn.FLAG_SCAN_CHUNKS):
+        p.flags = f
+        assert vdn.lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size)) == 0
+    p.flags = vdn.FLAG_SCAN_FRAMES | vdn.FLAG_SCAN_CHUNKS
+    rc = vdn.lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
+    assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"

@@ -508,3 +508,73 @@ def test_boundary_states_tensor_core(over, beta_tok):
     eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
     print(f"states {over}: F {eF:.2e} G {eG:.2e}")
     assert eF <= 1e-4 and eG <= 1e-4
+
+
+# (name, overrides, make_inputs kwargs, extra kwargs)
+SCAN_CASES = [
+    ("tiny_f32", None, {}, {}),
+    ("d64", dict(T=23, N=96, d=64, H=2), dict(alpha_range=(0.9, 1.0)), {}),
+    ("d128", dict(T=12, N=136, d=128, H=2), dict(alpha_range=(0.9, 1.0)), {}),
+    ("T1", dict(T=1, N=40), {}, {}),
+    ("T2", dict(T=2, N=24), {}, {}),
+    ("T7_partial_chunk", dict(T=7, N=5), dict(alpha_range=(0.85, 1.0)), {}),
+    ("chunk1_r0", dict(T=9, N=130, chunk=1, window_radius=0), {}, {}),
+    ("c3_r2", dict(T=12, N=64, chunk=3, window_radius=2), {}, {}),
+    ("text_full", dict(T=16, N=64), {}, dict(text_full=True)),
+    ("beta_per_token_d128", dict(T=8, N=40, d=128, H=2, n_text=37),
+     dict(beta_per_token=True), dict(beta_per_token=True)),
+    ("frozen_d64", dict(T=14, N=72), None, dict(frozen_state=True)),
+]
+
+
+@pytest.mark.parametrize("scan", ["frames", "chunks"])
+@pytest.mark.parametrize("name,over,mk,kw", SCAN_CASES, ids=[c[0] for c in SCAN_CASES])
+def test_scan_paths_match_the_oracle(name, over, mk, kw, scan):
+    """The two evaluations of the bidirectional scan (over frames, or chunk
+    composition + chunk scan) give the oracle's chunk-boundary states and
+    linear readout, on the tensor-core and FP32 frame kernels."""
+    if over is None and name == "tiny_f32":
+        cfg = CONFIGS["tiny_f32"]
+    else:
+        cfg = _edge_cfg(over)
+    if kw.get("frozen_state"):
+        inp = _frozen_inputs(cfg)
+    else:
+        inp = make_inputs(cfg, **mk)
+    d = to_dev(inp)
+    F, G = vdn.vda_boundary_states(d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], cfg.T,
+                                   alpha=d["alpha"], chunk=cfg.chunk,
+                                   window_radius=cfg.window_radius, scan=scan, **kw)
+    _, o_l = _branches(d, cfg, want_soft=False, scan=scan, **kw)
+    torch.cuda.synchronize()
+    okw = dict(text_full=kw.get("text_full", False), beta_per_token=kw.get("beta_per_token", False),
+               frozen=kw.get("frozen_state", False))
+    Fo, Go = O.boundary_states(inp["k"], inp["v"], inp["beta"], inp["text_k"], inp["text_v"],
+                               cfg.T, cfg.N, cfg.chunk, cfg.window_radius, alpha=inp["alpha"],
+                               **okw)
+    _, _, wl = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius, **okw)
+    tol = 1e-5 if cfg.dtype == "f32" else 1e-4
+    eF, eG = rel_err(F.double().cpu(), Fo), rel_err(G.double().cpu(), Go)
+    eL = rel_err(o_l.double().cpu(), wl)
+    print(f"scan={scan} {name}: F {eF:.2e} G {eG:.2e} o_lin {eL:.2e}")
+    assert eF <= tol and eG <= tol and eL <= tol
+
+
+def test_scan_paths_agree_on_the_768p_forward():
+    """At 768p the shape picks the frame scan.  The linear readout (FP32, before
+    any rounding) of the frame scan and of the chunk composition agree to FP32
+    rounding; the outputs, which pass through one fp16 rounding of the gated
+    operand (where a last-bit difference in o_lin can flip a rounding), agree
+    within the output tolerance."""
+    cfg = CONFIGS["768p_h4_bf16"]
+    d = to_dev(make_inputs(cfg, alpha_range=(0.9, 1.0)))
+    _, la = _branches(d, cfg, want_soft=False, scan="frames")
+    _, lb = _branches(d, cfg, want_soft=False, scan="chunks")
+    a = _fwd(d, cfg, scan="frames")
+    b = _fwd(d, cfg, scan="chunks")
+    torch.cuda.synchronize()
+    e_lin = float((la - lb).abs().max()) / float(lb.pow(2).mean().sqrt())
+    e_out = float((a - b).abs().max()) / float(b.float().pow(2).mean().sqrt())
+    print(f"768p (4 heads) frames vs chunks: o_lin {e_lin:.2e}, out {e_out:.2e}")
+    assert e_lin <= 1e-5
+    assert e_out <= TOL_OUT["bf16"]
