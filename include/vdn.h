@@ -209,6 +209,41 @@ VDN_API vdn_status vdn_hybrid_attn_fwd_split(const vdn_params *p, const void *q,
                                      size_t workspace_bytes, vdn_stream_t stream,
                                      const vdn_stage_events *ev);
 
+/* ---- The forward in two halves (head-sharded, Ulysses-style execution) -----
+ * The implementation section of the paper shards VDA by attention head over
+ * GPUs (Ulysses).  Every step of the forward is independent per head except
+ * the output projection, which contracts over heads.  These two calls split
+ * the forward at that point, so that a rank can compute the operand of its
+ * heads, exchange it (an all-to-all from head shards to token shards), and
+ * project its own tokens with the whole W:
+ *   vdn_hybrid_attn_fwd == vdn_hybrid_attn_operand + vdn_output_projection
+ * (bit for bit, on the same inputs).  Tensor-core path only (dtype BF16,
+ * d in {64, 128}, no VDN_FLAG_SIMT); otherwise VDN_ERR_UNSUPPORTED. */
+
+/* x: [B, L, 2, H, d_v] fp16 (IEEE binary16), caller-owned, 16-byte aligned:
+ *   x[b, l, 0, h, :] = g_s * o_s          (gated Softmax readout)
+ *   x[b, l, 1, h, :] = g_l * RMS(o_l)     (gated, RMS-normalised linear readout)
+ * i.e. the rows of the operand [g_s o_s | g_l RMS(o_l)] of the two output
+ * projections.  Other arguments, workspace and errors as vdn_hybrid_attn_fwd
+ * (W_o_* are not needed); values beyond the fp16 range set VDN_ERR_RANGE. */
+VDN_API vdn_status vdn_hybrid_attn_operand(const vdn_params *p, const void *q, const void *k,
+                                           const void *v, const float *beta, const float *alpha,
+                                           const void *text_k, const void *text_v,
+                                           const void *gates, void *x, void *workspace,
+                                           size_t workspace_bytes, vdn_stream_t stream);
+
+/* out[r, :] = x[r, 0, :, :] W_o_soft + x[r, 1, :, :] W_o_lin for r < rows:
+ * x [rows, 2, H, d_v] fp16 as vdn_hybrid_attn_operand writes it (any set of
+ * rows, e.g. one token shard holding every head), W_o_* [H*d_v, D_out] in
+ * params.dtype, out [rows, D_out] in params.out_dtype.  Only H, d, D_out, the
+ * dtypes and flags of `p` matter here (the rest is validated as usual); the
+ * workspace is one of vdn_workspace_bytes(p).  rows in 1 .. 2^30 (else
+ * VDN_ERR_SHAPE). */
+VDN_API vdn_status vdn_output_projection(const vdn_params *p, long long rows, const void *x,
+                                         const void *W_o_soft, const void *W_o_lin, void *out,
+                                         void *workspace, size_t workspace_bytes,
+                                         vdn_stream_t stream);
+
 /* ---- End to end from host memory ------------------------------------------
  * One forward whose inputs and output live in host memory: the call enqueues
  * the host -> device copies of every input, the forward, and the device ->

@@ -116,6 +116,10 @@ def lib() -> ctypes.CDLL:
                                                 ctypes.POINTER(ctypes.c_size_t)])
         L.vdn_host_slot_release.restype = ctypes.c_int
         L.vdn_host_slot_release.argtypes = [_P]
+        L.vdn_hybrid_attn_operand.restype = ctypes.c_int
+        L.vdn_hybrid_attn_operand.argtypes = [PP] + [_P] * 10 + [ctypes.c_size_t, _P]
+        L.vdn_output_projection.restype = ctypes.c_int
+        L.vdn_output_projection.argtypes = [PP, ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P]
         L.vdn_selftest_exp2.restype = ctypes.c_int
         L.vdn_selftest_exp2.argtypes = [_P, _P, ctypes.c_size_t, _P]
         _lib = L
@@ -236,6 +240,43 @@ def hybrid_attn_fwd(q, k, v, beta, text_k, text_v, W_soft, W_lin, gates, T, *, a
                                              _ptr(ws), ws.numel(), _stream(stream), ev)
     if rc != 0:
         raise VdnError(rc, "vdn_hybrid_attn_fwd")
+    return out
+
+
+def hybrid_attn_operand(q, k, v, beta, text_k, text_v, gates, T, *, alpha=None, x=None,
+                        workspace=None, stream=None, params=None, **kw):
+    """x float16 [B, L, 2, H, d]: the gated branch outputs [g_s*o_s, g_l*RMS(o_l)],
+    the operand of the output projections (vdn_hybrid_attn_operand)."""
+    import torch
+    p = params or params_for(q, v, text_k, T, **kw)
+    B, L, H, d = q.shape
+    if x is None:
+        x = torch.empty(B, L, 2, H, d, dtype=torch.float16, device=q.device)
+    ws = alloc_workspace(p, q.device) if workspace is None else workspace
+    rc = lib().vdn_hybrid_attn_operand(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                       _ptr(alpha), _ptr(text_k), _ptr(text_v), _ptr(gates),
+                                       _ptr(x), _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_hybrid_attn_operand")
+    return x
+
+
+def output_projection(x, W_soft, W_lin, params, *, out=None, workspace=None, stream=None):
+    """out [..., D_out] = x[..., 0, :, :] W_soft + x[..., 1, :, :] W_lin for an
+    operand x float16 [..., 2, H, d] (vdn_output_projection); ``params`` gives
+    H, d, D_out and the dtypes."""
+    import torch
+    p = params
+    lead = x.shape[:-3]
+    rows = int(x.numel() // (2 * p.H * p.d_k))
+    if out is None:
+        odt = torch.float32 if p.out_dtype == VDN_F32 else torch.bfloat16
+        out = torch.empty(*lead, p.D_out, dtype=odt, device=x.device)
+    ws = alloc_workspace(p, x.device) if workspace is None else workspace
+    rc = lib().vdn_output_projection(ctypes.byref(p), rows, _ptr(x), _ptr(W_soft), _ptr(W_lin),
+                                     _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_output_projection")
     return out
 
 

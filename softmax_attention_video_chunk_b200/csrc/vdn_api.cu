@@ -409,6 +409,60 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_params* p, const void* q, const void* k
                                     gates, out, workspace, workspace_bytes, stream, nullptr);
 }
 
+vdn_status vdn_hybrid_attn_operand(const vdn_params* p, const void* q, const void* k,
+                                   const void* v, const float* beta, const float* alpha,
+                                   const void* text_k, const void* text_v, const void* gates,
+                                   void* x, void* workspace, size_t workspace_bytes,
+                                   vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  if (!use_tc(*p)) return VDN_ERR_UNSUPPORTED;
+  VDN_TRY(common_inputs(p, q, k, v, beta, alpha, text_k, text_v, true));
+  VDN_TRY(check_ptr(gates, true));
+  VDN_TRY(check_ptr(x, true));
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  const WsLayout w = layout(*p);
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  VdaArgs va = vda_args(p, k, v, beta, alpha, text_k, text_v, ws);
+  AttnArgs aa = attn_args(p, q, k, v, text_k, text_v);
+  TcAttnArgs t = tc_attn_args(*p, aa, ws + w.vt, (int*)(ws + w.status));
+  // the fused Softmax and readout epilogues write straight into the caller's x
+  TcFwdArgs f = tc_fwd_args(*p, va, t, nullptr, nullptr, gates, nullptr, ws + w.wt, x);
+  f.q = q;
+  VDN_CUDA(launch_vda_states(va, st));
+  VDN_CUDA(launch_convert_v(t, st));
+  VDN_CUDA(launch_attn_tc(t, &f, nullptr, st));
+  VDN_CUDA(launch_readout_tc(f, st));
+  return VDN_OK;
+}
+
+vdn_status vdn_output_projection(const vdn_params* p, long long rows, const void* x,
+                                 const void* W_o_soft, const void* W_o_lin, void* out,
+                                 void* workspace, size_t workspace_bytes, vdn_stream_t stream) {
+  VDN_TRY(validate_params(p));
+  if (!use_tc(*p)) return VDN_ERR_UNSUPPORTED;
+  if (rows < 1 || rows > 2147483647LL / 2) return VDN_ERR_SHAPE;
+  VDN_TRY(check_ptr(x, true));
+  VDN_TRY(check_ptr(W_o_soft, true));
+  VDN_TRY(check_ptr(W_o_lin, true));
+  VDN_TRY(check_ptr(out, true));
+  VDN_TRY(check_ws(p, workspace, workspace_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  const WsLayout w = layout(*p);
+  VDN_CUDA(cudaMemsetAsync(ws, 0, 256, st));
+  TcFwdArgs f;
+  memset(&f, 0, sizeof(f));
+  f.B = 1; f.L = (int)rows; f.H = p->H; f.D = p->d_k; f.T = 1; f.N = (int)rows;
+  f.D_out = p->D_out; f.out_dtype = p->out_dtype; f.eps = p->rms_eps;
+  f.W_soft = W_o_soft; f.W_lin = W_o_lin; f.wt = (__half*)(ws + w.wt);
+  f.x = (__half*)const_cast<void*>(x); f.out = out; f.status = (int*)(ws + w.status);
+  VDN_CUDA(launch_convert_w(f, st));
+  VDN_CUDA(launch_gemm_tc(f, st));
+  return VDN_OK;
+}
+
 vdn_status vdn_hybrid_attn_fwd_host(const vdn_params* p, const vdn_host_inputs* hin,
                                     void* host_out, vdn_host_slot* slot, void* workspace,
                                     size_t workspace_bytes, vdn_stream_t copy_in,

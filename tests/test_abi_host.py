@@ -253,3 +253,33 @@ def test_scan_flags_are_exclusive():
     p.flags = vdn.FLAG_SCAN_FRAMES | vdn.FLAG_SCAN_CHUNKS
     rc = vdn.lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
     assert vdn.STATUS[rc] == "VDN_ERR_INVALID_ARG"
+
+
+def test_operand_and_projection_validate_before_launch():
+    L = vdn.lib()
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    need = vdn.workspace_bytes(p)
+    ws = 0x7f0000000000
+    ptr = [0x10000 + 0x1000 * i for i in range(10)]
+    # q k v beta alpha tk tv gates x
+    args = [ptr[0], ptr[1], ptr[2], ptr[3], None, ptr[4], ptr[5], ptr[6], ptr[7]]
+    bad = list(args)
+    bad[8] = None  # no operand buffer
+    assert vdn.STATUS[L.vdn_hybrid_attn_operand(ctypes.byref(p), *bad, ws, need, None)] == \
+        "VDN_ERR_INVALID_ARG"
+    bad = list(args)
+    bad[8] = ptr[7] + 8  # misaligned
+    assert vdn.STATUS[L.vdn_hybrid_attn_operand(ctypes.byref(p), *bad, ws, need, None)] == \
+        "VDN_ERR_ALIGNMENT"
+    ps = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", simt=True)
+    assert vdn.STATUS[L.vdn_hybrid_attn_operand(ctypes.byref(ps), *args, ws, need, None)] == \
+        "VDN_ERR_UNSUPPORTED"
+    pf = vdn.make_params(1, 2, 15, 16, 64, 8, "f32")
+    assert vdn.STATUS[L.vdn_output_projection(ctypes.byref(pf), 10, ptr[0], ptr[1], ptr[2],
+                                              ptr[3], ws, vdn.workspace_bytes(pf), None)] == \
+        "VDN_ERR_UNSUPPORTED"
+    for rows, code in ((0, "VDN_ERR_SHAPE"), (-5, "VDN_ERR_SHAPE"), (1 << 31, "VDN_ERR_SHAPE")):
+        assert vdn.STATUS[L.vdn_output_projection(ctypes.byref(p), rows, ptr[0], ptr[1], ptr[2],
+                                                  ptr[3], ws, need, None)] == code
+    assert vdn.STATUS[L.vdn_output_projection(ctypes.byref(p), 10, ptr[0], None, ptr[2],
+                                              ptr[3], ws, need, None)] == "VDN_ERR_INVALID_ARG"

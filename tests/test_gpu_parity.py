@@ -232,18 +232,67 @@ def test_text_query_rows_768p_sampled():
     assert e <= 2e-3
 
 
-def test_ulysses_one_rank_runs_the_library_forward():
-    """The head-sharded wrapper with its default per-rank forward (the CUDA
-    library) on one rank is the plain forward."""
+@pytest.mark.parametrize("P", [2, 4])
+def test_head_shards_through_the_library(P):
+    """The head-sharded forward on one GPU: P head shards run one after another
+    through vdn_hybrid_attn_operand (each with its heads' inputs), their
+    operands are put together as the head -> token all-to-all would, and
+    vdn_output_projection projects every token shard with the whole W.  Heads
+    are independent up to the projection, so this equals the plain forward bit
+    for bit, and the oracle within the output tolerance."""
     from softmax_attention_video_chunk_b200 import ulysses
-    cfg = _edge_cfg(dict(T=10, N=48))
-    d = to_dev(make_inputs(cfg))
-    args = (d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"], d["W_soft"],
-            d["W_lin"], d["gates"], cfg.T)
-    a = ulysses.ulysses_forward(*args)
-    b = vdn.hybrid_attn_fwd(*args)
+    cfg = _edge_cfg(dict(T=11, N=96, d=128, H=4, n_text=24))
+    inp = make_inputs(cfg, alpha_range=(0.9, 1.0), gates="random")
+    d = to_dev(inp)
+    H = cfg.H
+    x = torch.empty(cfg.B, cfg.L, 2, H, cfg.d, dtype=torch.float16, device="cuda")
+    for r in range(P):
+        hs = ulysses.head_slice(P, r, H)
+        b_h, a_h, tk_h, tv_h = ulysses.head_inputs(d["beta"], d["alpha"], d["text_k"],
+                                                    d["text_v"], hs)
+        xr = vdn.hybrid_attn_operand(d["q"][:, :, hs].contiguous(), d["k"][:, :, hs].contiguous(),
+                                     d["v"][:, :, hs].contiguous(), b_h, tk_h, tv_h,
+                                     d["gates"][:, :, :, hs].contiguous(), cfg.T, alpha=a_h)
+        x[:, :, :, hs] = xr
+    # token-sharded projection: rank r projects tokens [r L/P, (r+1) L/P)
+    p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"])
+    Ls = cfg.L // P
+    out = torch.cat([vdn.output_projection(x[:, r * Ls:(r + 1) * Ls].contiguous(), d["W_soft"],
+                                           d["W_lin"], p) for r in range(P)], dim=1)
+    plain = _fwd(d, cfg)
     torch.cuda.synchronize()
-    assert torch.equal(a, b)
+    assert torch.equal(out, plain)
+    want, _, _ = oracle_forward(inp, cfg.T, cfg.N, cfg.chunk, cfg.window_radius)
+    e = rel_err(out.double().cpu(), want)
+    print(f"head shards P={P}: {e:.2e}")
+    assert e <= TOL_OUT["bf16"]
+
+
+def test_operand_then_projection_is_the_forward():
+    """vdn_hybrid_attn_operand followed by vdn_output_projection is
+    vdn_hybrid_attn_fwd, bit for bit (text keys in the Softmax, per-token
+    write gates, random gates)."""
+    cfg = _edge_cfg(dict(T=9, N=130, d=128, H=2, n_text=77))
+    inp = make_inputs(cfg, gates="random", beta_per_token=True)
+    d = to_dev(inp)
+    kw = dict(text_softmax=True, beta_per_token=True)
+    x = vdn.hybrid_attn_operand(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
+                                d["gates"], cfg.T, **kw)
+    p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], **kw)
+    out = vdn.output_projection(x, d["W_soft"], d["W_lin"], p)
+    plain = _fwd(d, cfg, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, plain)
+    # the operand itself: x[..., 0] = g_s o_s, x[..., 1] = g_l RMS(o_l) (fp16)
+    o_s, o_l = _branches(d, cfg, **kw)
+    torch.cuda.synchronize()
+    g = d["gates"].float()
+    xs = (g[0] * o_s).to(torch.float16)
+    rms = o_l.pow(2).mean(dim=-1, keepdim=True).add(1e-6).rsqrt()
+    xl = (g[1] * o_l * rms).to(torch.float16)
+    for got, ref in ((x[:, :, 0], xs), (x[:, :, 1], xl)):
+        err = (got.float() - ref.float()).abs().max() / ref.float().pow(2).mean().sqrt()
+        assert float(err) <= 4e-3, float(err)
 
 
 @pytest.mark.parametrize("simt", [False, True])
