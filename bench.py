@@ -191,6 +191,8 @@ def base_line(args, cfg, value, ms_per_step, n_gpus):
                    "text_keys_in_softmax": bool(getattr(args, "text_softmax", False)),
                    "write_gate": "per token" if getattr(args, "beta_per_token", False)
                                  else "per frame",
+                   "projection": "MXFP8 (E4M3, 32-element UE8M0 blocks, FP32 accumulation)"
+                                 if getattr(args, "proj_mxfp8", False) else "fp16 operands",
                    "frame_rule": "frozen-state (comparison)"
                                  if getattr(args, "frozen_state", False) else "VDA",
                    "linear_feature_map": "VDA-Prep in the step (3x3 spatial + 5-tap temporal "
@@ -267,7 +269,8 @@ def run_ours(args, cfg):
         d["k"] = (d["k"].float() / float(cfg.N) ** 0.5).to(d["k"].dtype)
     p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], chunk=cfg.chunk,
                        window_radius=cfg.window_radius, text_softmax=args.text_softmax,
-                       beta_per_token=args.beta_per_token, frozen_state=args.frozen_state)
+                       beta_per_token=args.beta_per_token, frozen_state=args.frozen_state,
+                       proj_mxfp8=args.proj_mxfp8)
     ws = vdn.alloc_workspace(p)
     out = torch.empty(cfg.B, cfg.L, p.D_out, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -455,6 +458,8 @@ def main():
                     help="frame updates by the frozen-state comparison rule instead of VDA")
     ap.add_argument("--prep", action="store_true",
                     help="time VDA-Prep (linear-branch feature map of raw q, k, v) in every step")
+    ap.add_argument("--proj-mxfp8", action="store_true",
+                    help="output projections in MXFP8 (block-scaled E4M3, FP32 accumulation)")
     ap.add_argument("--alpha", action="store_true",
                     help="channel-wise decay gate alpha ~ U[0.9, 1] instead of none")
     args = ap.parse_args()

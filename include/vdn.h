@@ -123,6 +123,18 @@ typedef struct CUstream_st *vdn_stream_t;
  * one of them (setting both is VDN_ERR_INVALID_ARG). */
 #define VDN_FLAG_SCAN_FRAMES (1u << 5)
 #define VDN_FLAG_SCAN_CHUNKS (1u << 6)
+/* Reduced-precision mode of the output projections (implementation section:
+ * MXFP8 for the output GEMM): the fp16 operands x = [g_s o_s | g_l RMS(o_l)]
+ * and [W_o_soft; W_o_lin] are quantised to MXFP8 -- blocks of 32 elements
+ * along the contraction dimension share a power-of-two scale 2^e,
+ * e = floor(log2 max|v|) - 8 (stored as e + 127), elements v / 2^e rounded to
+ * E4M3 (ties to even, saturating at +-448) -- and multiplied on the block-
+ * scaled fp8 tensor cores with FP32 accumulation.  Tensor-core path only
+ * (else VDN_ERR_UNSUPPORTED).  Its error against the exact projection is that
+ * of the format (about 4% of the output RMS, up to about 25% at single
+ * outputs), far above the default path's; see vdn_mxfp8_quantize for the
+ * exact quantisation. */
+#define VDN_FLAG_PROJ_MXFP8 (1u << 7)
 
 typedef struct vdn_params {
   int B;             /* batch */
@@ -178,10 +190,11 @@ typedef struct vdn_stage_events {
 
 /* Same computation and arguments as vdn_hybrid_attn_fwd, and records
  * events[0] before the first kernel and events[i] after stage i on `stream`:
- * 1 VDA state path (frame statistics + solve, chunk composition, chunk scan),
- * 2 operand conversion (V^T and W^T to fp16; empty on the CUDA-core path),
- * 3 window+anchor Softmax, 4 linear readout (+ RMS norm and gate on the
- * tensor-core path), 5 output projection.  Used for live per-stage timing
+ * 1 VDA state path (frame statistics + solve, then the bidirectional scan),
+ * 2 V^T conversion to fp16 (empty on the CUDA-core path), 3 window+anchor
+ * Softmax, 4 linear readout (+ RMS norm and gate on the tensor-core path),
+ * 5 output projection (W^T conversion, with VDN_FLAG_PROJ_MXFP8 the MXFP8
+ * quantisation of both operands, and the GEMM).  Used for live per-stage timing
  * with cudaEventElapsedTime.  `ev` may be NULL (no events). */
 VDN_API vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params *p, const void *q, const void *k,
                                       const void *v, const float *beta, const float *alpha,
@@ -243,6 +256,23 @@ VDN_API vdn_status vdn_output_projection(const vdn_params *p, long long rows, co
                                          const void *W_o_soft, const void *W_o_lin, void *out,
                                          void *workspace, size_t workspace_bytes,
                                          vdn_stream_t stream);
+
+/* MXFP8 quantisation (the VDN_FLAG_PROJ_MXFP8 rule) of a row-major fp16
+ * (IEEE binary16) matrix x [rows, cols], cols a multiple of 128, in blocks of
+ * 32 along each row:
+ *  - codes [rows, cols] uint8: the E4M3 elements (1 sign, 4 exponent bits of
+ *    bias 7, 3 mantissa bits);
+ *  - scales: the shared exponents e + 127 (UE8M0) in 512-byte atoms, one per
+ *    128 rows x 128 columns: scale of row r, block j (columns 32j .. 32j+31) at
+ *    byte ((r / 128) * (cols / 128) + j / 4) * 512 + 16 (r % 32)
+ *    + 4 ((r % 128) / 32) + j % 4.  scales_bytes must hold
+ *    ceil(rows_padded / 128) * (cols / 128) * 512 bytes; rows in
+ *    [rows, rows_padded) get the smallest scale (e = -127).
+ * This is the layout the block-scaled tensor cores read.  Device pointers,
+ * 16-byte aligned; asynchronous on `stream`. */
+VDN_API vdn_status vdn_mxfp8_quantize(const void *x, long long rows, long long rows_padded,
+                                      int cols, void *codes, void *scales, size_t scales_bytes,
+                                      vdn_stream_t stream);
 
 /* ---- End to end from host memory ------------------------------------------
  * One forward whose inputs and output live in host memory: the call enqueues

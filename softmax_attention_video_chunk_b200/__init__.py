@@ -18,6 +18,7 @@ VDN_F32, VDN_BF16 = 0, 1
 FLAG_TEXT_FULL, FLAG_SIMT, FLAG_TEXT_SOFTMAX, FLAG_BETA_PER_TOKEN = 1, 2, 4, 8
 FLAG_FROZEN_STATE = 16
 FLAG_SCAN_FRAMES, FLAG_SCAN_CHUNKS = 32, 64
+FLAG_PROJ_MXFP8 = 128
 
 STATUS = {
     0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_SHAPE", 3: "VDN_ERR_DTYPE",
@@ -120,6 +121,9 @@ def lib() -> ctypes.CDLL:
         L.vdn_hybrid_attn_operand.argtypes = [PP] + [_P] * 10 + [ctypes.c_size_t, _P]
         L.vdn_output_projection.restype = ctypes.c_int
         L.vdn_output_projection.argtypes = [PP, ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P]
+        L.vdn_mxfp8_quantize.restype = ctypes.c_int
+        L.vdn_mxfp8_quantize.argtypes = [_P, ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int,
+                                         _P, _P, ctypes.c_size_t, _P]
         L.vdn_selftest_exp2.restype = ctypes.c_int
         L.vdn_selftest_exp2.argtypes = [_P, _P, ctypes.c_size_t, _P]
         _lib = L
@@ -129,7 +133,8 @@ def lib() -> ctypes.CDLL:
 def make_params(B, H, T, N, d, n_text, dtype="bf16", *, chunk=5, window_radius=1,
                 D_out=None, out_dtype="f32", softmax_scale=0.0, rms_eps=1e-6,
                 text_full=False, simt=False, text_softmax=False,
-                beta_per_token=False, frozen_state=False, scan=None) -> VdnParams:
+                beta_per_token=False, frozen_state=False, scan=None,
+                proj_mxfp8=False) -> VdnParams:
     p = VdnParams()
     dt = {"f32": VDN_F32, "bf16": VDN_BF16}
     rc = lib().vdn_params_init(ctypes.byref(p), B, H, T, N, d, n_text, dt[dtype])
@@ -141,7 +146,8 @@ def make_params(B, H, T, N, d, n_text, dtype="bf16", *, chunk=5, window_radius=1
                (FLAG_TEXT_SOFTMAX if text_softmax else 0) |
                (FLAG_BETA_PER_TOKEN if beta_per_token else 0) |
                (FLAG_FROZEN_STATE if frozen_state else 0) |
-               {None: 0, "frames": FLAG_SCAN_FRAMES, "chunks": FLAG_SCAN_CHUNKS}[scan])
+               {None: 0, "frames": FLAG_SCAN_FRAMES, "chunks": FLAG_SCAN_CHUNKS}[scan] |
+               (FLAG_PROJ_MXFP8 if proj_mxfp8 else 0))
     size = ctypes.c_size_t(0)
     rc = lib().vdn_workspace_bytes(ctypes.byref(p), ctypes.byref(size))
     if rc != 0:
@@ -503,6 +509,24 @@ def device_status(p: Optional[VdnParams], workspace, stream=None) -> int:
 def selftest_bounded_wait(workspace, limit_us: int, stream=None) -> int:
     """Enqueue the bounded-wait self-test (a wait that nothing satisfies)."""
     return lib().vdn_selftest_bounded_wait(_ptr(workspace), int(limit_us), _stream(stream))
+
+
+def mxfp8_quantize(x, rows_padded=None, stream=None):
+    """(codes uint8 [rows, cols], scales uint8 [atoms * 512]) of an fp16 device
+    matrix x [rows, cols] (vdn_mxfp8_quantize; cols a multiple of 128)."""
+    import torch
+    if x.dtype != torch.float16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D float16 tensor")
+    rows, cols = x.shape
+    rp = rows if rows_padded is None else rows_padded
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    nbytes = ((rp + 127) // 128) * (cols // 128) * 512
+    scales = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    rc = lib().vdn_mxfp8_quantize(_ptr(x), rows, rp, cols, _ptr(codes), _ptr(scales), nbytes,
+                                  _stream(stream))
+    if rc != 0:
+        raise VdnError(rc, "vdn_mxfp8_quantize")
+    return codes, scales
 
 
 def selftest_exp2(x, stream=None):

@@ -74,6 +74,17 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* b
   return make_tmap_sw(map, dt, rank, base, dims, strides_bytes, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Row-major uint8 matrix [rows][cols] (cols a multiple of 16), 128-byte
+// swizzled boxes of box_rows x box_cols bytes: the E4M3 operand tiles.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                  uint32_t box_cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t str[1] = {cols};
+  const uint32_t box[2] = {box_cols, box_rows};
+  return make_tmap_sw(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, str, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Dense (unswizzled) boxes, laid out in shared memory in row-major box order.
 bool make_tmap_plain(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {

@@ -23,6 +23,7 @@ struct WsLayout {
   size_t status, Mf, Rf, CM, CR, FS, GS;   // VDA state path
   size_t o_s, o_l, rinv;                   // CUDA-core path intermediates
   size_t vt, wt, x;                        // tensor-core path operands
+  size_t xq, sfa, wq, sfb;                 // MXFP8 projection operands and scales
   size_t vda_end;                          // end of the VDA state-path prefix
   size_t total;
 };
@@ -53,6 +54,13 @@ static WsLayout layout(const vdn_params& p) {
     w.vt = take(s.vt_bytes);
     w.wt = take(s.wt_bytes);
     w.x = take(s.x_bytes);
+    if (p.flags & VDN_FLAG_PROJ_MXFP8) {
+      const size_t K = 2 * H * d, M = B * L, No = p.D_out;
+      w.xq = take(M * K);
+      w.sfa = take(mx_scale_bytes((long long)M, (int)K));
+      w.wq = take(No * K);
+      w.sfb = take(mx_scale_bytes((long long)((No + 255) / 256 * 256), (int)K));
+    }
   } else {
     w.o_s = take(B * L * H * d * sizeof(float));
     w.o_l = take(B * L * H * d * sizeof(float));
@@ -66,7 +74,8 @@ static vdn_status validate_params(const vdn_params* p) {
   if (p == nullptr) return VDN_ERR_INVALID_ARG;
   if (p->flags & ~(unsigned)(VDN_FLAG_TEXT_FULL | VDN_FLAG_SIMT | VDN_FLAG_TEXT_SOFTMAX |
                              VDN_FLAG_BETA_PER_TOKEN | VDN_FLAG_FROZEN_STATE |
-                             VDN_FLAG_SCAN_FRAMES | VDN_FLAG_SCAN_CHUNKS))
+                             VDN_FLAG_SCAN_FRAMES | VDN_FLAG_SCAN_CHUNKS |
+                             VDN_FLAG_PROJ_MXFP8))
     return VDN_ERR_INVALID_ARG;
   if ((p->flags & VDN_FLAG_SCAN_FRAMES) && (p->flags & VDN_FLAG_SCAN_CHUNKS))
     return VDN_ERR_INVALID_ARG;
@@ -139,6 +148,26 @@ static vdn_status check_ws(const vdn_params* p, const void* ws, size_t ws_bytes)
   do {                                                   \
     if ((expr) != cudaSuccess) return VDN_ERR_CUDA;      \
   } while (0)
+
+// The projection out = x [W_soft; W_lin] of f.B * f.L rows from the fp16
+// operand f.x and W^T (converted into f.wt here): fp16 tcgen05 GEMM, or with
+// VDN_FLAG_PROJ_MXFP8 both operands quantised to MXFP8 and the block-scaled
+// fp8 GEMM.
+static cudaError_t launch_projection(const vdn_params* p, const TcFwdArgs& f, char* ws,
+                                     const WsLayout& w, cudaStream_t st) {
+  cudaError_t e = launch_convert_w(f, st);
+  if (e != cudaSuccess) return e;
+  if (!(p->flags & VDN_FLAG_PROJ_MXFP8)) return launch_gemm_tc(f, st);
+  const long long M = (long long)f.B * f.L;
+  const int K = 2 * f.H * f.D, No = f.D_out;
+  uint8_t *xq = (uint8_t*)(ws + w.xq), *sfa = (uint8_t*)(ws + w.sfa);
+  uint8_t *wq = (uint8_t*)(ws + w.wq), *sfb = (uint8_t*)(ws + w.sfb);
+  if ((e = launch_mx_quant(f.x, xq, sfa, M, (M + 127) / 128 * 128, K, st)) != cudaSuccess)
+    return e;
+  if ((e = launch_mx_quant(f.wt, wq, sfb, No, (No + 255) / 256 * 256, K, st)) != cudaSuccess)
+    return e;
+  return launch_mx_gemm(xq, sfa, wq, sfb, f.out, f.out_dtype, (int)M, No, K, f.status, st);
+}
 
 static VdaArgs vda_args(const vdn_params* p, const void* k, const void* v, const float* beta,
                         const float* alpha, const void* text_k, const void* text_v, char* ws) {
@@ -315,6 +344,7 @@ static vdn_status fwd_impl(const vdn_params* p, const void* q, const void* k, co
                            void* out, void* workspace, size_t workspace_bytes,
                            vdn_stream_t stream, const vdn_stage_events* ev) {
   VDN_TRY(validate_params(p));
+  if ((p->flags & VDN_FLAG_PROJ_MXFP8) && !use_tc(*p)) return VDN_ERR_UNSUPPORTED;
   VDN_TRY(common_inputs(p, q, k, v, beta, alpha, text_k, text_v, true));
   VDN_TRY(check_ptr(q_l, true));
   VDN_TRY(check_ptr(k_l, true));
@@ -344,13 +374,12 @@ static vdn_status fwd_impl(const vdn_params* p, const void* q, const void* k, co
     VDN_CUDA(launch_vda_states(va, st));
     VDN_CUDA(mark(1));
     VDN_CUDA(launch_convert_v(t, st));
-    VDN_CUDA(launch_convert_w(f, st));
     VDN_CUDA(mark(2));
     VDN_CUDA(launch_attn_tc(t, &f, nullptr, st));
     VDN_CUDA(mark(3));
     VDN_CUDA(launch_readout_tc(f, st));
     VDN_CUDA(mark(4));
-    VDN_CUDA(launch_gemm_tc(f, st));
+    VDN_CUDA(launch_projection(p, f, ws, w, st));
     VDN_CUDA(mark(5));
     return VDN_OK;
   }
@@ -458,8 +487,11 @@ vdn_status vdn_output_projection(const vdn_params* p, long long rows, const void
   f.D_out = p->D_out; f.out_dtype = p->out_dtype; f.eps = p->rms_eps;
   f.W_soft = W_o_soft; f.W_lin = W_o_lin; f.wt = (__half*)(ws + w.wt);
   f.x = (__half*)const_cast<void*>(x); f.out = out; f.status = (int*)(ws + w.status);
-  VDN_CUDA(launch_convert_w(f, st));
-  VDN_CUDA(launch_gemm_tc(f, st));
+  if (p->flags & VDN_FLAG_PROJ_MXFP8) {
+    // the scale and code regions of the workspace are sized for B*T*N rows
+    if (rows > (long long)p->B * p->T * p->N) return VDN_ERR_WORKSPACE;
+  }
+  VDN_CUDA(launch_projection(p, f, ws, w, st));
   return VDN_OK;
 }
 
@@ -534,6 +566,21 @@ vdn_status vdn_hybrid_attn_fwd_host(const vdn_params* p, const vdn_host_inputs* 
   slot->used = 1;
   if (h2d_bytes != nullptr) *h2d_bytes = h2d;
   if (d2h_bytes != nullptr) *d2h_bytes = out_bytes;
+  return VDN_OK;
+}
+
+vdn_status vdn_mxfp8_quantize(const void* x, long long rows, long long rows_padded, int cols,
+                              void* codes, void* scales, size_t scales_bytes,
+                              vdn_stream_t stream) {
+  if (rows < 1 || rows_padded < rows || rows_padded > (1LL << 40) || cols < 128 ||
+      cols % 128 != 0)
+    return VDN_ERR_SHAPE;
+  VDN_TRY(check_ptr(x, true));
+  VDN_TRY(check_ptr(codes, true));
+  VDN_TRY(check_ptr(scales, true));
+  if (scales_bytes < mx_scale_bytes(rows_padded, cols)) return VDN_ERR_WORKSPACE;
+  VDN_CUDA(launch_mx_quant((const __half*)x, (uint8_t*)codes, (uint8_t*)scales, rows,
+                           rows_padded, cols, (cudaStream_t)stream));
   return VDN_OK;
 }
 

@@ -58,4 +58,12 @@ cudaError_t launch_attn_tc(const TcAttnArgs& t, const TcFwdArgs* fused, float* o
 cudaError_t launch_readout_tc(const TcFwdArgs& f, cudaStream_t st);
 cudaError_t launch_gemm_tc(const TcFwdArgs& f, cudaStream_t st);
 
+// MXFP8 projection (k_mxfp8.cu)
+size_t mx_scale_bytes(long long rows_padded, int cols);
+cudaError_t launch_mx_quant(const __half* x, uint8_t* codes, uint8_t* scales, long long rows,
+                            long long rows_padded, int cols, cudaStream_t st);
+cudaError_t launch_mx_gemm(const uint8_t* xq, const uint8_t* sfa, const uint8_t* wq,
+                           const uint8_t* sfb, void* out, vdn_dtype out_dtype, int M, int Nout,
+                           int K, int* status, cudaStream_t st);
+
 }  // namespace vdn

@@ -53,7 +53,7 @@ def test_params_init_defaults():
     ("chunk", 0, "VDN_ERR_SHAPE"), ("window_radius", -1, "VDN_ERR_SHAPE"),
     ("n_text", -1, "VDN_ERR_SHAPE"), ("D_out", 12, "VDN_ERR_SHAPE"),
     ("d_v", 32, "VDN_ERR_UNSUPPORTED"), ("dtype", 7, "VDN_ERR_DTYPE"),
-    ("out_dtype", 3, "VDN_ERR_DTYPE"), ("flags", 1 << 7, "VDN_ERR_INVALID_ARG"),
+    ("out_dtype", 3, "VDN_ERR_DTYPE"), ("flags", 1 << 8, "VDN_ERR_INVALID_ARG"),
     ("softmax_scale", -1.0, "VDN_ERR_INVALID_ARG"), ("rms_eps", float("nan"), "VDN_ERR_INVALID_ARG"),
 ])
 def test_param_validation(field, value, code):
@@ -283,3 +283,29 @@ def test_operand_and_projection_validate_before_launch():
                                                   ptr[3], ws, need, None)] == code
     assert vdn.STATUS[L.vdn_output_projection(ctypes.byref(p), 10, ptr[0], None, ptr[2],
                                               ptr[3], ws, need, None)] == "VDN_ERR_INVALID_ARG"
+
+
+def test_mxfp8_quantize_validates():
+    L = vdn.lib()
+    x, c, s = 0x10000, 0x20000, 0x30000
+    need = 1 * 2 * 512  # 100 rows padded to 128, 256 columns
+    for rows, rp, cols, code in ((0, 0, 256, "VDN_ERR_SHAPE"), (100, 99, 256, "VDN_ERR_SHAPE"),
+                                 (100, 128, 200, "VDN_ERR_SHAPE"), (100, 128, 64, "VDN_ERR_SHAPE")):
+        assert vdn.STATUS[L.vdn_mxfp8_quantize(x, rows, rp, cols, c, s, need, None)] == code
+    assert vdn.STATUS[L.vdn_mxfp8_quantize(x, 100, 128, 256, c, s, need - 1, None)] == \
+        "VDN_ERR_WORKSPACE"
+    assert vdn.STATUS[L.vdn_mxfp8_quantize(x + 8, 100, 128, 256, c, s, need, None)] == \
+        "VDN_ERR_ALIGNMENT"
+
+
+def test_mxfp8_projection_needs_the_tensor_core_path():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "f32", proj_mxfp8=True)
+    need = vdn.workspace_bytes(p)
+    ptrs = [0x10000 + 0x1000 * i for i in range(11)]
+    ptrs[4] = None
+    rc = vdn.lib().vdn_hybrid_attn_fwd(ctypes.byref(p), *ptrs, 0x7f0000000000, need, None)
+    assert vdn.STATUS[rc] == "VDN_ERR_UNSUPPORTED"
+    # the workspace grows by the quantised operands and their scales
+    a = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16"))
+    b = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", proj_mxfp8=True))
+    assert b > a
