@@ -32,58 +32,77 @@ size_t mx_scale_bytes(long long rows_padded, int cols) {
   return (size_t)((rows_padded + 127) / 128) * (size_t)(cols / 128) * 512u;
 }
 
-// One warp per (row, 128-column chunk): lane l holds columns 4l .. 4l+3 of
-// the chunk; the 8 lanes of a 32-column block share its maximum by shuffles.
-// Rows in [rows, rows_padded) write the smallest scale only (their elements
-// are never read: the GEMM's loads of them come back as zeros).
+// Each lane quantises 8 consecutive elements (one 16-byte load, one 8-byte
+// store); the 4 lanes of a 32-element block share its maximum by shuffles, so
+// a warp covers 256 columns (two scale atoms' worth of one row).  Grid-stride
+// over (row, 256-column piece).  Rows in [rows, rows_padded) write the
+// smallest scale only (their elements are never read: the GEMM's loads of them
+// come back as zeros).
 __global__ void __launch_bounds__(256)
 mx_quant_rows_kernel(const __half* __restrict__ x, uint8_t* __restrict__ codes,
                      uint8_t* __restrict__ scales, long long rows, long long rows_padded,
                      int cols) {
   const int lane = threadIdx.x & 31;
-  const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int chunks = cols / 128;
-  if (wid >= rows_padded * chunks) return;  // uniform over the warp
-  const long long r = wid / chunks;
-  const int ch = (int)(wid % chunks);
-  const bool live = r < rows;
-  float v[4] = {0.f, 0.f, 0.f, 0.f};
-  if (live) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(x + r * cols + ch * 128 + 4 * lane);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    const float2 a = __half22float2(h2[0]), b = __half22float2(h2[1]);
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-  }
-  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-  // e = floor(log2 amax) - 8 from the exponent field (amax, from fp16 values,
-  // is a normal float32 or zero)
-  int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 8 : -127;
-  e = max(-127, min(127, e));
-  const float inv = ldexpf(1.f, -e);  // exact power of two
-  if (live) {
-    uint32_t packed = 0;
+  const int chunks = cols / 128;        // 128-column scale atoms per row
+  const int pieces = (cols + 255) / 256;
+  const long long nwork = rows_padded * pieces;
+  const long long wstride = (long long)gridDim.x * 8;
+  for (long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); w < nwork; w += wstride) {
+    const long long r = w / pieces;
+    const int col = (int)(w % pieces) * 256 + 8 * lane;
+    const bool in_cols = col < cols;  // uniform per 32-element block (cols % 128 == 0)
+    const bool live = r < rows && in_cols;
+    float v[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_fp8_storage_t q = __nv_cvt_float_to_fp8(v[i] * inv, __NV_SATFINITE, __NV_E4M3);
-      packed |= (uint32_t)q << (8 * i);
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    if (live) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(x + r * cols + col);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
     }
-    *reinterpret_cast<uint32_t*>(codes + r * cols + ch * 128 + 4 * lane) = packed;
-  }
-  if ((lane & 7) == 0) {
-    const int blk = lane >> 3;  // block of the chunk (0..3): the byte in the atom
-    const size_t atom = (size_t)(r / 128) * (size_t)chunks + (size_t)ch;
-    scales[atom * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + blk] = (uint8_t)(e + 127);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    // e = floor(log2 amax) - 8 from the exponent field (amax, from fp16
+    // values, is a normal float32 or zero)
+    int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 8 : -127;
+    e = max(-127, min(127, e));
+    const float inv = ldexpf(1.f, -e);  // exact power of two
+    if (live) {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo |= (uint32_t)__nv_cvt_float_to_fp8(v[i] * inv, __NV_SATFINITE, __NV_E4M3) << (8 * i);
+        hi |= (uint32_t)__nv_cvt_float_to_fp8(v[4 + i] * inv, __NV_SATFINITE, __NV_E4M3)
+              << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(codes + r * cols + col) = make_uint2(lo, hi);
+    }
+    if ((lane & 3) == 0 && in_cols) {
+      const int j = col / 32;  // block index along the row
+      const size_t atom = (size_t)(r / 128) * (size_t)chunks + (size_t)(j / 4);
+      scales[atom * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + (j % 4)] = (uint8_t)(e + 127);
+    }
   }
 }
 
+int sm_count();
+
 cudaError_t launch_mx_quant(const __half* x, uint8_t* codes, uint8_t* scales, long long rows,
                             long long rows_padded, int cols, cudaStream_t st) {
-  const long long warps = rows_padded * (cols / 128);
-  mx_quant_rows_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(x, codes, scales, rows,
-                                                                    rows_padded, cols);
+  const long long warps = rows_padded * ((cols + 255) / 256);
+  long long blocks = (warps + 7) / 8;
+  const long long cap = (long long)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  mx_quant_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, codes, scales, rows, rows_padded,
+                                                         cols);
   return cudaGetLastError();
 }
 
@@ -298,8 +317,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   ptx::tc_fence_after();
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
-
-int sm_count();
 
 // xq [M][K], wq [Nout][K] E4M3; sfa for M rows padded to 128, sfb for Nout
 // rows padded to 256 (two atoms per 256-column output tile).
