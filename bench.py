@@ -75,6 +75,12 @@ ATTN_TRAFFIC_PER_HEAD = (1001.119e6 + 113.169152e6) / 4
 ATTN_TRAFFIC_SHAPES = {(75, 1536, 128)}
 
 
+# B200 datasheet figures (dense bf16 tensor throughput, HBM3e bandwidth):
+# context for the fractions, which are also given against the measured peaks.
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 7700.0
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -392,19 +398,29 @@ def run_ours(args, cfg):
             "bound": "tensor", "kernel": "attn_tc_kernel (window+anchor Softmax)",
             "achieved": achieved, "peak": pk["tc_sust"], "unit": "TFLOP/s",
             "frac": achieved / pk["tc_sust"],
+            "frac_of_burst_peak": achieved / pk["tc"],
+            "frac_of_datasheet_peak": achieved / DATASHEET_BF16_TFLOPS,
             "traffic": (ATTN_TRAFFIC_PER_HEAD * cfg.B * cfg.H
                         if (cfg.T, cfg.N, cfg.d) in ATTN_TRAFFIC_SHAPES else None),
             "traffic_note": "ncu capture of the 4-head 768p shape, scaled by heads",
             "peak_kind": f"{pk['src']} bf16 dense, sustained (kernel timed inside the step loop)",
             "algorithmic_flops_per_launch": wm["f_soft"], "ms_per_launch": soft_ms,
         }
+        # the whole forward against the larger of FLOPs / tensor peak and bytes
+        # / HBM bandwidth: the headline fraction, given against the measured
+        # burst and sustained peaks and the datasheet ones
+        def path_frac(tc, hbm):
+            return 1e3 * max(wm["f_total"] / (tc * 1e12), wm["bytes_min"] / (hbm * 1e9)) / ms_per_step
         line["path_roofline"] = {
             "flops": wm["f_total"], "bytes_min": wm["bytes_min"],
             "t_roofline_ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms_per_step,
             "peak_tflops": pk["tc"], "peak_hbm_gbs": pk["hbm"], "peaks": pk["src"] + " (burst)",
+            "frac_of_sustained_peak": path_frac(pk["tc_sust"], pk["hbm"]),
+            "frac_of_datasheet_peak": path_frac(DATASHEET_BF16_TFLOPS, DATASHEET_HBM_GBS),
+            "datasheet_peaks": {"bf16_tflops": DATASHEET_BF16_TFLOPS, "hbm_gbs": DATASHEET_HBM_GBS},
         }
         line["stages_ms"] = dict(zip(vdn.STAGE_NAMES, [round(x, 4) for x in stage_ms]))
-        line["gpu_launches"] = args.steps * ((8 if vdn.use_tc_params(p) else 6) +
+        line["gpu_launches"] = args.steps * (vdn.forward_launches(p) +
                                              (2 if prep_ms is not None else 0))
         if tq_ms is not None:
             line["stages_ms"]["text_rows"] = round(tq_ms, 4)

@@ -182,6 +182,19 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const
                                const void *gates, void *out, void *workspace,
                                size_t workspace_bytes, vdn_stream_t stream);
 
+/* Number of kernel launches that vdn_hybrid_attn_fwd enqueues for `p`
+ * (host only; the status-word clear is a memset, not counted).  The state
+ * path takes 2 kernels (frame statistics + solve, then the direct scan over
+ * frames) or 3 (frame statistics + solve, chunk composition, chunk scan): the
+ * library picks the route from the shape and the device's SM count unless
+ * VDN_FLAG_SCAN_FRAMES / VDN_FLAG_SCAN_CHUNKS forces it.  Then, on the
+ * tensor-core path: V^T conversion, Softmax, readout, W^T conversion and the
+ * GEMM (with VDN_FLAG_PROJ_MXFP8: two quantisations and the block-scaled
+ * GEMM); on the CUDA-core path: Softmax, readout, RMS factors, projection.
+ * Validates `p` like the compute calls; `launches` must not be NULL
+ * (VDN_ERR_INVALID_ARG). */
+VDN_API vdn_status vdn_forward_launches(const vdn_params *p, int *launches);
+
 /* Stage boundaries recorded by vdn_hybrid_attn_fwd_staged. */
 #define VDN_STAGES 5 /* VDA states, operand conversion, Softmax, readout, projection */
 typedef struct vdn_stage_events {

@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.vdn_params_init.argtypes = [PP] + [ctypes.c_int] * 7
         L.vdn_workspace_bytes.restype = ctypes.c_int
         L.vdn_workspace_bytes.argtypes = [PP, ctypes.POINTER(ctypes.c_size_t)]
+        L.vdn_forward_launches.restype = ctypes.c_int
+        L.vdn_forward_launches.argtypes = [PP, ctypes.POINTER(ctypes.c_int)]
         L.vdn_hybrid_attn_fwd.restype = ctypes.c_int
         L.vdn_hybrid_attn_fwd.argtypes = [PP] + [_P] * 12 + [ctypes.c_size_t, _P]
         L.vdn_hybrid_attn_fwd_staged.restype = ctypes.c_int
@@ -161,6 +163,15 @@ def workspace_bytes(p: VdnParams) -> int:
     if rc != 0:
         raise VdnError(rc, "vdn_workspace_bytes")
     return size.value
+
+
+def forward_launches(p: VdnParams) -> int:
+    """Kernel launches that one ``hybrid_attn_fwd`` call enqueues for ``p``."""
+    n = ctypes.c_int(0)
+    rc = lib().vdn_forward_launches(ctypes.byref(p), ctypes.byref(n))
+    if rc != 0:
+        raise VdnError(rc, "vdn_forward_launches")
+    return n.value
 
 
 # --------------------------------------------------------------------------

@@ -549,6 +549,24 @@ vda_readout_kernel(const TIn* __restrict__ q, const float* __restrict__ alpha,
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
+// Chunk composition + chunk scan, or the direct frame scan: whichever the
+// wave-count model puts first (or the one a.scan_mode forces).  Sequential
+// steps per CTA: composition 2 (C - 1) products then nc scan steps; direct
+// scan T products.  CTAs: the composition runs 2 B H nc (D / 32) of them,
+// both scans 2 B H (D / 32); two CTAs per SM.
+bool vda_frame_scan_route(const VdaArgs& a) {
+  if (a.scan_mode != 0) return a.scan_mode == 1;
+  const long long nc = (a.T + a.C - 1) / a.C;
+  const long long slots = 2LL * sm_count();
+  const long long cta_scan = 2LL * a.B * a.H * (a.D / 32);
+  const long long cta_comp = cta_scan * nc;
+  const long long waves_scan = (cta_scan + slots - 1) / slots;
+  const long long waves_comp = (cta_comp + slots - 1) / slots;
+  const long long cost_chunk = waves_comp * 2LL * (a.C - 1) + waves_scan * nc;
+  const long long cost_direct = waves_scan * (long long)a.T;
+  return cost_direct <= cost_chunk;
+}
+
 template <int D, typename TIn>
 static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
   const int H = a.H, B = a.B, T = a.T, nc = (a.T + a.C - 1) / a.C;
@@ -565,19 +583,7 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
         a.alpha, a.Mf, a.Rf, H, T, a.N, a.n_text, a.beta_tok, a.frozen);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // Chunk composition + chunk scan, or the direct frame scan: whichever the
-  // wave-count model puts first.  Sequential steps per CTA: composition
-  // 2 (C - 1) products then nc scan steps; direct scan T products.  CTAs: the
-  // composition runs 2 B H nc (D / 32) of them, both scans 2 B H (D / 32);
-  // two CTAs per SM.
-  const long long slots = 2LL * sm_count();
-  const long long cta_scan = 2LL * B * H * (D / 32);
-  const long long cta_comp = cta_scan * nc;
-  const long long waves_scan = (cta_scan + slots - 1) / slots;
-  const long long waves_comp = (cta_comp + slots - 1) / slots;
-  const long long cost_chunk = waves_comp * 2LL * (a.C - 1) + waves_scan * nc;
-  const long long cost_direct = waves_scan * (long long)T;
-  if (a.scan_mode == 1 || (a.scan_mode == 0 && cost_direct <= cost_chunk)) {
+  if (vda_frame_scan_route(a)) {
     const size_t sm = sizeof(float) * ((size_t)D * (D + 4) + (size_t)D * 32);
     auto kern = vda_frame_scan_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

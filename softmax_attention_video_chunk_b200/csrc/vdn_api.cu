@@ -693,6 +693,23 @@ vdn_status vdn_text_query_attn(const vdn_params* p, const void* text_q, const vo
   return VDN_OK;
 }
 
+vdn_status vdn_forward_launches(const vdn_params* p, int* launches) {
+  VDN_TRY(validate_params(p));
+  if (launches == nullptr) return VDN_ERR_INVALID_ARG;
+  if ((p->flags & VDN_FLAG_PROJ_MXFP8) && !use_tc(*p)) return VDN_ERR_UNSUPPORTED;
+  VdaArgs va;
+  memset(&va, 0, sizeof(va));
+  va.B = p->B; va.H = p->H; va.T = p->T; va.D = p->d_k; va.C = p->chunk;
+  va.scan_mode = (p->flags & VDN_FLAG_SCAN_FRAMES) ? 1 : ((p->flags & VDN_FLAG_SCAN_CHUNKS) ? 2 : 0);
+  int n = vda_frame_scan_route(va) ? 2 : 3;
+  if (use_tc(*p))
+    n += 4 + ((p->flags & VDN_FLAG_PROJ_MXFP8) ? 3 : 1);
+  else
+    n += 4;
+  *launches = n;
+  return VDN_OK;
+}
+
 vdn_status vdn_device_status(const vdn_params* p, void* workspace, vdn_stream_t stream) {
   if (p != nullptr) VDN_TRY(validate_params(p));
   if (workspace == nullptr) return VDN_ERR_WORKSPACE;

@@ -26,6 +26,9 @@ struct VdaArgs {
 cudaError_t launch_frame_tc(const VdaArgs& a, cudaStream_t st);
 
 cudaError_t launch_vda_states(const VdaArgs& a, cudaStream_t st);
+// true: launch_vda_states runs the direct frame scan (2 kernels in all);
+// false: chunk composition + chunk scan (3 kernels in all)
+bool vda_frame_scan_route(const VdaArgs& a);
 cudaError_t launch_vda_readout_simt(const VdaArgs& a, const void* q, float* o_l, cudaStream_t st);
 cudaError_t launch_gather_boundary(const VdaArgs& a, float* F, float* G, cudaStream_t st);
 

@@ -309,3 +309,36 @@ def test_mxfp8_projection_needs_the_tensor_core_path():
     a = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16"))
     b = vdn.workspace_bytes(vdn.make_params(1, 2, 15, 16, 64, 8, "bf16", proj_mxfp8=True))
     assert b > a
+
+
+@pytest.mark.parametrize("shape,dtype,flags,expect", [
+    # 768p: 24 heads, 75 frames: the direct frame scan (75 sequential products
+    # in one wave against 10 waves of composition + 15 scan steps)
+    ((1, 24, 75, 1536, 128, 512), "bf16", 0, 7),
+    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_SCAN_CHUNKS, 8),
+    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_SCAN_FRAMES, 7),
+    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_PROJ_MXFP8, 9),
+    # few heads, 15 frames: composition fits one wave, so chunks win (8 + 3 < 15)
+    ((1, 2, 15, 16, 64, 8), "bf16", 0, 8),
+    # one chunk: the frame scan (2 products) beats composition (8 + 1)
+    ((1, 2, 2, 16, 64, 8), "bf16", 0, 7),
+    # CUDA-core path: states (2 or 3), Softmax, readout, RMS factors, projection
+    ((1, 24, 75, 1536, 128, 512), "f32", 0, 6),
+    ((1, 2, 15, 16, 64, 8), "bf16", vdn.FLAG_SIMT, 7),
+])
+def test_forward_launch_count(shape, dtype, flags, expect):
+    p = vdn.make_params(*shape, dtype)
+    p.flags |= flags
+    assert vdn.forward_launches(p) == expect
+
+
+def test_forward_launch_count_validates():
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "bf16")
+    assert vdn.STATUS[vdn.lib().vdn_forward_launches(ctypes.byref(p), None)] == "VDN_ERR_INVALID_ARG"
+    p.chunk = 0
+    with pytest.raises(vdn.VdnError):
+        vdn.forward_launches(p)
+    p = vdn.make_params(1, 2, 15, 16, 64, 8, "f32")
+    p.flags |= vdn.FLAG_PROJ_MXFP8
+    with pytest.raises(vdn.VdnError):
+        vdn.forward_launches(p)
