@@ -129,8 +129,11 @@ typedef struct CUstream_st *vdn_stream_t;
  * along the contraction dimension share a power-of-two scale 2^e,
  * e = floor(log2 max|v|) - 8 (stored as e + 127), elements v / 2^e rounded to
  * E4M3 (ties to even, saturating at +-448) -- and multiplied on the block-
- * scaled fp8 tensor cores with FP32 accumulation.  Tensor-core path only
- * (else VDN_ERR_UNSUPPORTED).  Its error against the exact projection is that
+ * scaled fp8 tensor cores with FP32 accumulation.  In the forward, the
+ * Softmax and readout epilogues quantise their rows of x in registers (the
+ * same fp16 values, the same codes and scales as vdn_mxfp8_quantize), so x
+ * never reaches memory in fp16; vdn_output_projection quantises the x it is
+ * given.  Tensor-core path only (else VDN_ERR_UNSUPPORTED).  Its error against the exact projection is that
  * of the format (about 4% of the output RMS, up to about 25% at single
  * outputs), far above the default path's; see vdn_mxfp8_quantize for the
  * exact quantisation. */
@@ -189,8 +192,9 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const
  * library picks the route from the shape and the device's SM count unless
  * VDN_FLAG_SCAN_FRAMES / VDN_FLAG_SCAN_CHUNKS forces it.  Then, on the
  * tensor-core path: V^T conversion, Softmax, readout, W^T conversion and the
- * GEMM (with VDN_FLAG_PROJ_MXFP8: two quantisations and the block-scaled
- * GEMM); on the CUDA-core path: Softmax, readout, RMS factors, projection.
+ * GEMM (with VDN_FLAG_PROJ_MXFP8: the quantisation of W^T and the block-
+ * scaled GEMM, x arriving quantised from the epilogues); on the CUDA-core
+ * path: Softmax, readout, RMS factors, projection.
  * Validates `p` like the compute calls; `launches` must not be NULL
  * (VDN_ERR_INVALID_ARG). */
 VDN_API vdn_status vdn_forward_launches(const vdn_params *p, int *launches);
@@ -207,7 +211,7 @@ typedef struct vdn_stage_events {
  * 2 V^T conversion to fp16 (empty on the CUDA-core path), 3 window+anchor
  * Softmax, 4 linear readout (+ RMS norm and gate on the tensor-core path),
  * 5 output projection (W^T conversion, with VDN_FLAG_PROJ_MXFP8 the MXFP8
- * quantisation of both operands, and the GEMM).  Used for live per-stage timing
+ * quantisation of W^T, and the GEMM; x is quantised inside stages 3 and 4).  Used for live per-stage timing
  * with cudaEventElapsedTime.  `ev` may be NULL (no events). */
 VDN_API vdn_status vdn_hybrid_attn_fwd_staged(const vdn_params *p, const void *q, const void *k,
                                       const void *v, const float *beta, const float *alpha,

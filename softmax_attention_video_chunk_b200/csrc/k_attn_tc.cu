@@ -26,6 +26,7 @@
 // its MMAs and copies, frees TMEM and exits.
 #include <math.h>
 
+#include "mx_encode.cuh"
 #include "tc_ptx.cuh"
 #include "vdn_common.cuh"
 #include "vdn_tc.h"
@@ -127,7 +128,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                const __grid_constant__ CUtensorMap map_tk,
                const __grid_constant__ CUtensorMap map_tvt, int n_text, Geo geo, int B, int H,
                float scale_log2, const __nv_bfloat16* __restrict__ gates,
-               __half* __restrict__ x, float* __restrict__ o_s, int* __restrict__ status,
+               __half* __restrict__ x, uint8_t* __restrict__ xq, uint8_t* __restrict__ sfa,
+               float* __restrict__ o_s, int* __restrict__ status,
                int n_qtext, int kv_split, float* __restrict__ ml) {
   constexpr int BM = 128, NS = 2;
   constexpr int QT = BM * D * 2;   // bytes of a Q tile
@@ -471,22 +473,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
           if (!valid) continue;
           if constexpr (FUSED) {
             const uint4* gp = reinterpret_cast<const uint4*>(gates + (tok * H + h) * D + 32 * c);
-            uint4* xp = reinterpret_cast<uint4*>(x + tok * (size_t)(2 * H * D) + (size_t)h * D + 32 * c);
+            uint32_t hw[16];  // g_s * o_s of this 32-column block, fp16
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
               const uint4 gg = gp[v4];
               const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gg);
-              uint4 outv;
-              uint32_t* ow = reinterpret_cast<uint32_t*>(&outv);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float2 gf = __bfloat1622float2(g2[e]);
                 const float a0 = gf.x * __uint_as_float(o[8 * v4 + 2 * e]) * inv;
                 const float a1 = gf.y * __uint_as_float(o[8 * v4 + 2 * e + 1]) * inv;
                 bad |= !(fabsf(a0) <= 65504.f) || !(fabsf(a1) <= 65504.f);
-                ow[e] = pack_half2(a0, a1);
+                hw[4 * v4 + e] = pack_half2(a0, a1);
               }
-              xp[v4] = outv;
+            }
+            const size_t K = (size_t)(2 * H * D);
+            if (xq == nullptr) {
+              uint4* xp = reinterpret_cast<uint4*>(x + tok * K + (size_t)h * D + 32 * c);
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4)
+                xp[v4] = make_uint4(hw[4 * v4], hw[4 * v4 + 1], hw[4 * v4 + 2], hw[4 * v4 + 3]);
+            } else {  // the same fp16 values, quantised to MXFP8 (one 32-element block)
+              uint32_t cw[8];
+              const uint32_t eb = mx::encode32(hw, cw);
+              uint4* qp = reinterpret_cast<uint4*>(xq + tok * K + (size_t)h * D + 32 * c);
+              qp[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+              qp[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+              sfa[mx::sf_offset(tok, (h * D + 32 * c) / 32, (int)K)] = (uint8_t)eb;
             }
           } else {
             float4* op = reinterpret_cast<float4*>(o_out + (tok * H + h) * D + 32 * c);
@@ -598,7 +611,8 @@ static cudaError_t launch_attn_t(const TcAttnArgs& t, const TcFwdArgs* f, float*
   const unsigned grid = (unsigned)pairs * (unsigned)(t.B * t.H);
   kern<<<grid, 320, sm, st>>>(mq, mk, mv, mtk, mtv, t.n_text_keys, geo, t.B, t.H, scale_log2,
                               FUSED ? (const __nv_bfloat16*)f->gates : nullptr,
-                              FUSED ? f->x : nullptr, kv_split > 1 ? t.part : o_s, t.status,
+                              FUSED ? f->x : nullptr, FUSED ? f->xq : nullptr,
+                              FUSED ? f->sfa : nullptr, kv_split > 1 ? t.part : o_s, t.status,
                               n_qtext, kv_split, t.ml);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (kv_split > 1) {

@@ -19,6 +19,7 @@
 #include <cuda_fp8.h>
 #include <math.h>
 
+#include "mx_encode.cuh"
 #include "tc_ptx.cuh"
 #include "vdn_common.cuh"
 #include "vdn_tc.h"
@@ -43,7 +44,6 @@ mx_quant_rows_kernel(const __half* __restrict__ x, uint8_t* __restrict__ codes,
                      uint8_t* __restrict__ scales, long long rows, long long rows_padded,
                      int cols) {
   const int lane = threadIdx.x & 31;
-  const int chunks = cols / 128;        // 128-column scale atoms per row
   const int pieces = (cols + 255) / 256;
   const long long nwork = rows_padded * pieces;
   const long long wstride = (long long)gridDim.x * 8;
@@ -70,26 +70,15 @@ mx_quant_rows_kernel(const __half* __restrict__ x, uint8_t* __restrict__ codes,
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    // e = floor(log2 amax) - 8 from the exponent field (amax, from fp16
-    // values, is a normal float32 or zero)
-    int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 8 : -127;
-    e = max(-127, min(127, e));
-    const float inv = ldexpf(1.f, -e);  // exact power of two
+    const int e = mx::block_exp(amax);
+    const float inv = mx::inv_scale(e);
     if (live) {
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo |= (uint32_t)__nv_cvt_float_to_fp8(v[i] * inv, __NV_SATFINITE, __NV_E4M3) << (8 * i);
-        hi |= (uint32_t)__nv_cvt_float_to_fp8(v[4 + i] * inv, __NV_SATFINITE, __NV_E4M3)
-              << (8 * i);
-      }
+      const uint32_t lo = mx::e4m3x2(v[0] * inv, v[1] * inv) | (mx::e4m3x2(v[2] * inv, v[3] * inv) << 16);
+      const uint32_t hi = mx::e4m3x2(v[4] * inv, v[5] * inv) | (mx::e4m3x2(v[6] * inv, v[7] * inv) << 16);
       *reinterpret_cast<uint2*>(codes + r * cols + col) = make_uint2(lo, hi);
     }
-    if ((lane & 3) == 0 && in_cols) {
-      const int j = col / 32;  // block index along the row
-      const size_t atom = (size_t)(r / 128) * (size_t)chunks + (size_t)(j / 4);
-      scales[atom * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + (j % 4)] = (uint8_t)(e + 127);
-    }
+    if ((lane & 3) == 0 && in_cols)  // block index along the row: col / 32
+      scales[mx::sf_offset((size_t)r, col / 32, cols)] = (uint8_t)(e + 127);
   }
 }
 

@@ -21,6 +21,7 @@
 //               operand x.
 #include <math.h>
 
+#include "mx_encode.cuh"
 #include "tc_ptx.cuh"
 #include "vdn_common.cuh"
 #include "vdn_tc.h"
@@ -35,7 +36,8 @@ __global__ void __launch_bounds__(192, 2)
 readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __restrict__ alpha,
                   const float* __restrict__ Rf, const float* __restrict__ FS,
                   const float* __restrict__ GS, const __nv_bfloat16* __restrict__ gl,
-                  __half* __restrict__ x, int H, int T, int N, int C, int R, float init_scale,
+                  __half* __restrict__ x, uint8_t* __restrict__ xq, uint8_t* __restrict__ sfa,
+                  int H, int T, int N, int C, int R, float init_scale,
                   float eps, int* __restrict__ status) {
   constexpr int BM = 128;
   constexpr int QT = BM * D * 2;      // bytes of a q tile
@@ -186,14 +188,11 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
         ptx::tmem_wait_ld();
         if (!valid) continue;
         const uint4* gp = reinterpret_cast<const uint4*>(gl + (row * H + h) * D + 32 * cc);
-        uint4* xp = reinterpret_cast<uint4*>(x + row * (size_t)(2 * H * D) + (size_t)H * D +
-                                             (size_t)h * D + 32 * cc);
+        uint32_t hw[16];  // g_l * RMS(o_l) of this 32-column block, fp16
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
           const uint4 gg = gp[v4];
           const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gg);
-          uint4 ov;
-          uint32_t* ow = reinterpret_cast<uint32_t*>(&ov);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 gv = __bfloat1622float2(g2[e]);
@@ -201,9 +200,22 @@ readout_tc_kernel(const __grid_constant__ CUtensorMap map_q, const float* __rest
             const float y1 = gv.y * __uint_as_float(r[8 * v4 + 2 * e + 1]) * rinv;
             bad |= !(fabsf(y0) <= 65504.f) || !(fabsf(y1) <= 65504.f);
             __half2 hv = __floats2half2_rn(y0, y1);
-            ow[e] = *reinterpret_cast<uint32_t*>(&hv);
+            hw[4 * v4 + e] = *reinterpret_cast<uint32_t*>(&hv);
           }
-          xp[v4] = ov;
+        }
+        const size_t K = (size_t)(2 * H * D), col = (size_t)H * D + (size_t)h * D + 32 * cc;
+        if (xq == nullptr) {
+          uint4* xp = reinterpret_cast<uint4*>(x + row * K + col);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            xp[v4] = make_uint4(hw[4 * v4], hw[4 * v4 + 1], hw[4 * v4 + 2], hw[4 * v4 + 3]);
+        } else {  // the same fp16 values, quantised to MXFP8 (one 32-element block)
+          uint32_t cw[8];
+          const uint32_t eb = mx::encode32(hw, cw);
+          uint4* qp = reinterpret_cast<uint4*>(xq + row * K + col);
+          qp[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          qp[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          sfa[mx::sf_offset(row, (int)(col / 32), (int)K)] = (uint8_t)eb;
         }
       }
       ptx::tc_fence_before();
@@ -232,7 +244,8 @@ static cudaError_t launch_t(const TcFwdArgs& f, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const __nv_bfloat16* gl = (const __nv_bfloat16*)f.gates + (size_t)f.B * f.L * f.H * f.D;
-  kern<<<dim3(a.T, a.H, a.B), 192, sm, st>>>(mq, a.alpha, a.Rf, a.FS, a.GS, gl, f.x, a.H, a.T,
+  kern<<<dim3(a.T, a.H, a.B), 192, sm, st>>>(mq, a.alpha, a.Rf, a.FS, a.GS, gl, f.x, f.xq, f.sfa,
+                                             a.H, a.T,
                                              a.N, a.C, a.R, a.init_scale, f.eps, f.status);
   return cudaGetLastError();
 }

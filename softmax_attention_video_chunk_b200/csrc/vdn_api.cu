@@ -152,7 +152,7 @@ static vdn_status check_ws(const vdn_params* p, const void* ws, size_t ws_bytes)
 // The projection out = x [W_soft; W_lin] of f.B * f.L rows from the fp16
 // operand f.x and W^T (converted into f.wt here): fp16 tcgen05 GEMM, or with
 // VDN_FLAG_PROJ_MXFP8 both operands quantised to MXFP8 and the block-scaled
-// fp8 GEMM.
+// fp8 GEMM.  With f.xq set, the epilogues have already written x in MXFP8.
 static cudaError_t launch_projection(const vdn_params* p, const TcFwdArgs& f, char* ws,
                                      const WsLayout& w, cudaStream_t st) {
   cudaError_t e = launch_convert_w(f, st);
@@ -162,7 +162,8 @@ static cudaError_t launch_projection(const vdn_params* p, const TcFwdArgs& f, ch
   const int K = 2 * f.H * f.D, No = f.D_out;
   uint8_t *xq = (uint8_t*)(ws + w.xq), *sfa = (uint8_t*)(ws + w.sfa);
   uint8_t *wq = (uint8_t*)(ws + w.wq), *sfb = (uint8_t*)(ws + w.sfb);
-  if ((e = launch_mx_quant(f.x, xq, sfa, M, (M + 127) / 128 * 128, K, st)) != cudaSuccess)
+  if (f.xq == nullptr &&
+      (e = launch_mx_quant(f.x, xq, sfa, M, (M + 127) / 128 * 128, K, st)) != cudaSuccess)
     return e;
   if ((e = launch_mx_quant(f.wt, wq, sfb, No, (No + 255) / 256 * 256, K, st)) != cudaSuccess)
     return e;
@@ -371,6 +372,18 @@ static vdn_status fwd_impl(const vdn_params* p, const void* q, const void* k, co
     TcAttnArgs t = tc_attn_args(*p, aa, ws + w.vt, (int*)(ws + w.status));
     TcFwdArgs f = tc_fwd_args(*p, va, t, W_o_soft, W_o_lin, gates, out, ws + w.wt, ws + w.x);
     f.q = q_l;  // the readout's queries
+    if (p->flags & VDN_FLAG_PROJ_MXFP8) {
+      // the Softmax and readout epilogues write x in MXFP8; scale bytes of
+      // the rows past B*L in the last 128-row group read as the smallest scale
+      f.xq = (uint8_t*)(ws + w.xq);
+      f.sfa = (uint8_t*)(ws + w.sfa);
+      const long long M = (long long)f.B * f.L;
+      const int K = 2 * f.H * f.D;
+      if (M % 128 != 0) {
+        const size_t group = (size_t)(K / 128) * 512u;
+        VDN_CUDA(cudaMemsetAsync(f.sfa + (size_t)(M / 128) * group, 0, group, st));
+      }
+    }
     VDN_CUDA(launch_vda_states(va, st));
     VDN_CUDA(mark(1));
     VDN_CUDA(launch_convert_v(t, st));
@@ -703,7 +716,7 @@ vdn_status vdn_forward_launches(const vdn_params* p, int* launches) {
   va.scan_mode = (p->flags & VDN_FLAG_SCAN_FRAMES) ? 1 : ((p->flags & VDN_FLAG_SCAN_CHUNKS) ? 2 : 0);
   int n = vda_frame_scan_route(va) ? 2 : 3;
   if (use_tc(*p))
-    n += 4 + ((p->flags & VDN_FLAG_PROJ_MXFP8) ? 3 : 1);
+    n += 4 + ((p->flags & VDN_FLAG_PROJ_MXFP8) ? 2 : 1);
   else
     n += 4;
   *launches = n;

@@ -37,6 +37,11 @@ struct TcFwdArgs {
   const void *W_soft, *W_lin;  // bf16 [H*D][D_out]
   __half* wt;                  // fp16 [D_out][2*H*D]
   __half* x;                   // fp16 [B*L][2*H*D] = [g_s*o_s | g_l*RMS(o_l)]
+  // MXFP8 projection: when xq != nullptr the Softmax and readout epilogues
+  // write x as E4M3 codes [B*L][2*H*D] and its UE8M0 scales (atom layout of
+  // mx_scale_bytes) instead of fp16
+  uint8_t* xq = nullptr;
+  uint8_t* sfa = nullptr;
   void* out;                   // [B*L][D_out]
   const void* q;
   VdaArgs vda;

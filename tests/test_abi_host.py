@@ -317,7 +317,7 @@ def test_mxfp8_projection_needs_the_tensor_core_path():
     ((1, 24, 75, 1536, 128, 512), "bf16", 0, 7),
     ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_SCAN_CHUNKS, 8),
     ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_SCAN_FRAMES, 7),
-    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_PROJ_MXFP8, 9),
+    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_PROJ_MXFP8, 8),
     # few heads, 15 frames: composition fits one wave, so chunks win (8 + 3 < 15)
     ((1, 2, 15, 16, 64, 8), "bf16", 0, 8),
     # one chunk: the frame scan (2 products) beats composition (8 + 1)

@@ -121,16 +121,23 @@ def test_mxfp8_forward_within_the_formats_bounds(name, over, mk):
     assert not torch.equal(out, plain)
 
 
-def test_mxfp8_operand_projection_entry():
-    """vdn_output_projection with the flag is the MXFP8 half of the forward."""
-    cfg = _cfg(dict(T=9, N=130, H=2, d=128, n_text=40))
-    d = to_dev(make_inputs(cfg, gates="random"))
+@pytest.mark.parametrize("name,over,mk", CASES, ids=[c[0] for c in CASES])
+def test_mxfp8_operand_projection_entry(name, over, mk):
+    """vdn_output_projection with the flag is the MXFP8 half of the forward:
+    the forward's Softmax and readout epilogues quantise their fp16 rows in
+    registers, the entry quantises the fp16 operand with the stand-alone
+    quantiser, and the two give the same codes and scales (bit-equal outputs),
+    including the scale rows past B*L in the last 128-row group (d64_H3 has
+    936 rows)."""
+    cfg = _cfg(over)
+    d = to_dev(make_inputs(cfg, **mk))
     p = vdn.params_for(d["q"], d["v"], d["text_k"], cfg.T, d["W_soft"], proj_mxfp8=True)
     x = vdn.hybrid_attn_operand(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                                d["gates"], cfg.T, params=p)
+                                d["gates"], cfg.T, alpha=d["alpha"], params=p)
     out = vdn.output_projection(x, d["W_soft"], d["W_lin"], p)
     fwd = vdn.hybrid_attn_fwd(d["q"], d["k"], d["v"], d["beta"], d["text_k"], d["text_v"],
-                              d["W_soft"], d["W_lin"], d["gates"], cfg.T, params=p)
+                              d["W_soft"], d["W_lin"], d["gates"], cfg.T, alpha=d["alpha"],
+                              params=p)
     torch.cuda.synchronize()
     assert torch.equal(out, fwd)
 
