@@ -29,7 +29,14 @@ namespace vdn {
 int sm_count();
 
 // ---------------------------------------------------------------------------
-// S1 + S2: frame statistics and Gauss-Jordan solve
+// S1 + S2: frame statistics and Gauss-Jordan solve.
+// Per-frame maps (both frame kernels write the same): for video frame t,
+// Mf[1 + t] = X_t and Rf[1 + t] = W_t, with X_t = (I + beta A_t)^-1 and the
+// update S_t = X_t (Diag(alpha_t) S_{t-1} + W_t) (VDA), or X_t = I - beta A_t
+// and S_t = X_t Diag(alpha_t) S_{t-1} + W_t (frozen-state rule); anchor
+// frames write X = I, W = 0 (S_t = Diag(alpha_t) S_{t-1} under both).  The
+// text virtual frame writes Mf[0] = X_0 and its state Rf[0] = X_0 W_0 (VDA)
+// or W_0 (frozen).
 // ---------------------------------------------------------------------------
 template <int D, typename TIn>
 __global__ void __launch_bounds__(256)
@@ -49,12 +56,11 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
   float* Mo = Mout + (bh * (T + 1) + f) * mat;
   float* Ro = Rout + (bh * (T + 1) + f) * mat;
   const int t = f - 1;
-  const float* al = (alpha != nullptr && f >= 1) ? alpha + (bh * T + t) * D : nullptr;
 
-  if (f >= 1 && (t == 0 || t == T - 1)) {  // anchor: decay only, no write
+  if (f >= 1 && (t == 0 || t == T - 1)) {  // anchor: no write (X = I, W = 0)
     for (int e = tid; e < D * D; e += blockDim.x) {
       const int i = e / D, j = e % D;
-      Mo[e] = (i == j) ? (al ? al[i] : 1.f) : 0.f;
+      Mo[e] = (i == j) ? 1.f : 0.f;
       Ro[e] = 0.f;
     }
     return;
@@ -125,20 +131,23 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
     }
   }
   __syncthreads();
-  if (frozen) {  // frozen-state rule: M = (I - beta A) Diag(alpha), R = beta W
+  if (frozen) {  // frozen-state rule: X = I - beta A, W = beta W
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       const int i = ty * RT + r;
 #pragma unroll
       for (int m = 0; m < CT; ++m) {
         const int j = tx + 16 * m;
-        Mo[i * D + j] = ((i == j ? 1.f : 0.f) - bt * accA[r][m]) * (al ? al[j] : 1.f);
+        Mo[i * D + j] = (i == j ? 1.f : 0.f) - bt * accA[r][m];
         Ro[i * D + j] = bt * accW[r][m];
       }
     }
     return;
   }
-  // [I + beta A | Diag(alpha) | beta W]
+  // [I + beta A | I | beta W]; video frames write beta W now and eliminate
+  // the first two blocks only (-> X); the text frame also carries beta W
+  // through (-> X beta W, its state)
+  const int ncol = (f == 0) ? 3 * D : 2 * D;
 #pragma unroll
   for (int r = 0; r < RT; ++r) {
     const int i = ty * RT + r;
@@ -147,11 +156,12 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
       const int j = tx + 16 * m;
       aug[i * SD + j] = bt * accA[r][m] + (i == j ? 1.f : 0.f);
       aug[i * SD + 2 * D + j] = bt * accW[r][m];
+      if (f >= 1) Ro[i * D + j] = bt * accW[r][m];
     }
   }
   for (int e = tid; e < D * D; e += blockDim.x) {
     const int i = e / D, j = e % D;
-    aug[i * SD + D + j] = (i == j) ? (al ? al[i] : 1.f) : 0.f;
+    aug[i * SD + D + j] = (i == j) ? 1.f : 0.f;
   }
 
   // Gauss-Jordan without pivoting (I + A is symmetric positive definite with
@@ -163,16 +173,16 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
   for (int p = 0; p < D; ++p) {
     __syncthreads();
     const float inv = 1.f / aug[p * SD + p];
-    for (int j = p + tid; j < 3 * D; j += blockDim.x) prow[j] = aug[p * SD + j] * inv;
+    for (int j = p + tid; j < ncol; j += blockDim.x) prow[j] = aug[p * SD + j] * inv;
     for (int i = tid; i < D; i += blockDim.x) pcol[i] = aug[i * SD + p];
     __syncthreads();
     for (int i = warp; i < D; i += nwarps) {
       const float fi = pcol[i];
       float* row = aug + i * SD;
       if (i == p) {
-        for (int j = p + lane; j < 3 * D; j += 32) row[j] = prow[j];
+        for (int j = p + lane; j < ncol; j += 32) row[j] = prow[j];
       } else {
-        for (int j = p + lane; j < 3 * D; j += 32) row[j] = fmaf(-fi, prow[j], row[j]);
+        for (int j = p + lane; j < ncol; j += 32) row[j] = fmaf(-fi, prow[j], row[j]);
       }
     }
   }
@@ -180,21 +190,24 @@ vda_frame_solve_kernel(const TIn* __restrict__ k, const TIn* __restrict__ v,
   for (int e = tid; e < D * D; e += blockDim.x) {
     const int i = e / D, j = e % D;
     Mo[e] = aug[i * SD + D + j];
-    Ro[e] = aug[i * SD + 2 * D + j];
+    if (f == 0) Ro[e] = aug[i * SD + 2 * D + j];
   }
 }
 
 // ---------------------------------------------------------------------------
 // S3: chunk composition.  Forward: frames s..e-1 in increasing order;
-// reverse: e-1..s.  (M, R) <- (M_t M, M_t R + R_t).  Both products act on
-// columns independently, so each CTA composes one 32-column slice of M and R
-// (the whole M_t is staged once per frame).
+// reverse: e-1..s.  With M_t = X_t Diag(alpha_t):
+//   (M, R) <- (X_t (Diag(alpha_t) M), X_t (Diag(alpha_t) R + W_t))      VDA
+//   (M, R) <- (X_t (Diag(alpha_t) M), X_t (Diag(alpha_t) R) + W_t)      frozen
+// starting from the first frame's (X_t Diag(alpha_t), X_t W_t) (frozen: W_t).
+// Both products act on columns independently, so each CTA composes one
+// 32-column slice of M and R (the whole X_t is staged once per frame).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
 vda_chunk_compose_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf,
-                         float* __restrict__ CM, float* __restrict__ CR, int B, int H,
-                         int T, int C) {
+                         const float* __restrict__ alpha, float* __restrict__ CM,
+                         float* __restrict__ CR, int B, int H, int T, int C, bool frozen) {
   constexpr int RT = D / 32, SD = D + 1;
   const int cb = (blockIdx.x % (D / 32)) * 32;
   const int c = blockIdx.x / (D / 32);
@@ -206,46 +219,74 @@ vda_chunk_compose_kernel(const float* __restrict__ Mf, const float* __restrict__
   const size_t bh = (size_t)b * H + h;
   const int s = c * C, e = min(T, (c + 1) * C);
   extern __shared__ float smem[];
-  float* Mt = smem;            // [D][SD]
+  float* Mt = smem;            // [D][SD]  X_t
   float* Ma = Mt + D * SD;     // [D][32]  slice of the composed M
   float* Ra = Ma + D * 32;     // [D][32]  slice of the composed R
 
   const int nfr = e - s;
   for (int step = 0; step < nfr; ++step) {
     const int t = dir == 0 ? s + step : e - 1 - step;
-    const float* Mg = Mf + (bh * (T + 1) + 1 + t) * mat;
-    const float* Rg = Rf + (bh * (T + 1) + 1 + t) * mat;
+    const float* Xg = Mf + (bh * (T + 1) + 1 + t) * mat;
+    const float* Wg = Rf + (bh * (T + 1) + 1 + t) * mat;
+    const float* al = alpha != nullptr ? alpha + (bh * T + t) * D : nullptr;
     __syncthreads();
-    if (step == 0) {
-      for (int q = tid; q < D * 32; q += blockDim.x) {
-        const int i = q >> 5, j = q & 31;
-        Ma[q] = Mg[i * D + cb + j];
-        Ra[q] = Rg[i * D + cb + j];
+    for (int q = tid; q < D * D; q += blockDim.x) Mt[(q / D) * SD + (q % D)] = Xg[q];
+    // this thread's 4 x 4 block of the slices, before the products
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const int i = ty * RT + r;
+      const float ai = al != nullptr ? al[i] : 1.f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int j = tx * 4 + m;
+        const float w = Wg[i * D + cb + j];
+        if (step == 0) {  // M = X_t Diag(alpha_t) (no product); R pre-product = W_t
+          Ma[i * 32 + j] = Xg[i * D + cb + j] * (al != nullptr ? al[cb + j] : 1.f);
+          Ra[i * 32 + j] = w;
+        } else {
+          Ma[i * 32 + j] *= ai;
+          Ra[i * 32 + j] = frozen ? ai * Ra[i * 32 + j] : fmaf(ai, Ra[i * 32 + j], w);
+        }
       }
-      continue;
     }
-    for (int q = tid; q < D * D; q += blockDim.x) Mt[(q / D) * SD + (q % D)] = Mg[q];
+    if (step == 0 && frozen) continue;  // (X_t Diag(alpha_t), W_t): no product
     __syncthreads();
+    const bool do_m = step > 0;
     float am[RT][4], ar[RT][4];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
 #pragma unroll
       for (int m = 0; m < 4; ++m) am[r][m] = ar[r][m] = 0.f;
+    if (do_m) {
 #pragma unroll 4
-    for (int l = 0; l < D; ++l) {
-      const float4 bm = *reinterpret_cast<const float4*>(Ma + l * 32 + tx * 4);
-      const float4 br = *reinterpret_cast<const float4*>(Ra + l * 32 + tx * 4);
+      for (int l = 0; l < D; ++l) {
+        const float4 bm = *reinterpret_cast<const float4*>(Ma + l * 32 + tx * 4);
+        const float4 br = *reinterpret_cast<const float4*>(Ra + l * 32 + tx * 4);
 #pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const float a = Mt[(ty * RT + r) * SD + l];
-        am[r][0] = fmaf(a, bm.x, am[r][0]);
-        am[r][1] = fmaf(a, bm.y, am[r][1]);
-        am[r][2] = fmaf(a, bm.z, am[r][2]);
-        am[r][3] = fmaf(a, bm.w, am[r][3]);
-        ar[r][0] = fmaf(a, br.x, ar[r][0]);
-        ar[r][1] = fmaf(a, br.y, ar[r][1]);
-        ar[r][2] = fmaf(a, br.z, ar[r][2]);
-        ar[r][3] = fmaf(a, br.w, ar[r][3]);
+        for (int r = 0; r < RT; ++r) {
+          const float a = Mt[(ty * RT + r) * SD + l];
+          am[r][0] = fmaf(a, bm.x, am[r][0]);
+          am[r][1] = fmaf(a, bm.y, am[r][1]);
+          am[r][2] = fmaf(a, bm.z, am[r][2]);
+          am[r][3] = fmaf(a, bm.w, am[r][3]);
+          ar[r][0] = fmaf(a, br.x, ar[r][0]);
+          ar[r][1] = fmaf(a, br.y, ar[r][1]);
+          ar[r][2] = fmaf(a, br.z, ar[r][2]);
+          ar[r][3] = fmaf(a, br.w, ar[r][3]);
+        }
+      }
+    } else {  // first frame: the R product only
+#pragma unroll 4
+      for (int l = 0; l < D; ++l) {
+        const float4 br = *reinterpret_cast<const float4*>(Ra + l * 32 + tx * 4);
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const float a = Mt[(ty * RT + r) * SD + l];
+          ar[r][0] = fmaf(a, br.x, ar[r][0]);
+          ar[r][1] = fmaf(a, br.y, ar[r][1]);
+          ar[r][2] = fmaf(a, br.z, ar[r][2]);
+          ar[r][3] = fmaf(a, br.w, ar[r][3]);
+        }
       }
     }
     __syncthreads();
@@ -255,8 +296,8 @@ vda_chunk_compose_kernel(const float* __restrict__ Mf, const float* __restrict__
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int j = tx * 4 + m;
-        Ma[i * 32 + j] = am[r][m];
-        Ra[i * 32 + j] = ar[r][m] + Rg[i * D + cb + j];
+        if (do_m) Ma[i * 32 + j] = am[r][m];
+        Ra[i * 32 + j] = frozen ? ar[r][m] + Wg[i * D + cb + j] : ar[r][m];
       }
     }
   }
@@ -344,18 +385,20 @@ vda_chunk_scan_kernel(const float* __restrict__ Rf, const float* __restrict__ CM
 
 // ---------------------------------------------------------------------------
 // S3+S4 for short clips: the bidirectional scan run directly over the frames,
-// S <- M_t S + R_t, keeping only the chunk-boundary states (FS[k] after the
-// frames of chunks < k, GS[k] after the frames of chunks >= k).  It needs T
-// sequential steps instead of ceil(T / C), but does one product per frame
-// instead of the composition's two per frame plus the chunk scan, and reads
-// the per-frame maps directly.  Anchor frames (no write) only decay:
-// S <- Diag(alpha_t) S.  One CTA per 32-column slice of S and direction.
+// S <- X_t (Diag(alpha_t) S + W_t) (frozen-state rule: X_t Diag(alpha_t) S +
+// W_t), keeping only the chunk-boundary states (FS[k] after the frames of
+// chunks < k, GS[k] after the frames of chunks >= k).  It needs T sequential
+// steps instead of ceil(T / C), but does one product per frame instead of the
+// composition's two per frame plus the chunk scan, and reads the per-frame
+// maps directly.  Anchor frames (no write) only decay: S <- Diag(alpha_t) S.
+// One CTA per 32-column slice of S and direction.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf,
                       const float* __restrict__ alpha, float* __restrict__ FS,
-                      float* __restrict__ GS, int B, int H, int T, int C, float init_scale) {
+                      float* __restrict__ GS, int B, int H, int T, int C, float init_scale,
+                      bool frozen) {
   constexpr int RT = D / 32, SD = D + 4;  // row stride keeps float4 stores aligned
   const int cb = blockIdx.x * 32, h = blockIdx.y, b = blockIdx.z >> 1, dir = blockIdx.z & 1;
   const int nc = (T + C - 1) / C;
@@ -397,7 +440,7 @@ vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf
     const float* Rg = Rf + (bh * (T + 1) + 1 + t) * mat;
     float acc[RT][4];
     __syncthreads();
-    if (anchor) {  // M_t = Diag(alpha_t), R_t = 0
+    if (anchor) {  // X_t = I, W_t = 0
       const float* al = alpha != nullptr ? alpha + (bh * T + t) * D : nullptr;
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
@@ -408,6 +451,22 @@ vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf
       }
       if (step + 1 < T && !is_anchor(frame_of(step + 1))) load_m(frame_of(step + 1));
     } else {
+      // this thread's 4 x 4 block of the slice: Diag(alpha_t) S (+ W_t, VDA)
+      const float* al = alpha != nullptr ? alpha + (bh * T + t) * D : nullptr;
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        const int i = ty * RT + r;
+        const float a = al != nullptr ? al[i] : 1.f;
+        float4 sv = *reinterpret_cast<const float4*>(Ss + i * 32 + tx * 4);
+        if (frozen) {
+          sv.x *= a; sv.y *= a; sv.z *= a; sv.w *= a;
+        } else {
+          const float4 wv = *reinterpret_cast<const float4*>(Rg + i * D + cb + tx * 4);
+          sv.x = fmaf(a, sv.x, wv.x); sv.y = fmaf(a, sv.y, wv.y);
+          sv.z = fmaf(a, sv.z, wv.z); sv.w = fmaf(a, sv.w, wv.w);
+        }
+        *reinterpret_cast<float4*>(Ss + i * 32 + tx * 4) = sv;
+      }
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int q = tid + k * 256;
@@ -432,14 +491,16 @@ vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf
           acc[r][3] = fmaf(a, sv.w, acc[r][3]);
         }
       }
+      if (frozen) {
 #pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const int i = ty * RT + r;
-        const float4 rv = *reinterpret_cast<const float4*>(Rg + i * D + cb + tx * 4);
-        acc[r][0] += rv.x;
-        acc[r][1] += rv.y;
-        acc[r][2] += rv.z;
-        acc[r][3] += rv.w;
+        for (int r = 0; r < RT; ++r) {
+          const int i = ty * RT + r;
+          const float4 rv = *reinterpret_cast<const float4*>(Rg + i * D + cb + tx * 4);
+          acc[r][0] += rv.x;
+          acc[r][1] += rv.y;
+          acc[r][2] += rv.z;
+          acc[r][3] += rv.w;
+        }
       }
     }
     __syncthreads();
@@ -551,7 +612,7 @@ vda_readout_kernel(const TIn* __restrict__ q, const float* __restrict__ alpha,
 // ---------------------------------------------------------------------------
 // Chunk composition + chunk scan, or the direct frame scan: whichever the
 // wave-count model puts first (or the one a.scan_mode forces).  Sequential
-// steps per CTA: composition 2 (C - 1) products then nc scan steps; direct
+// steps per CTA: composition 2 C - 1 products then nc scan steps; direct
 // scan T products.  CTAs: the composition runs 2 B H nc (D / 32) of them,
 // both scans 2 B H (D / 32); two CTAs per SM.
 bool vda_frame_scan_route(const VdaArgs& a) {
@@ -562,7 +623,7 @@ bool vda_frame_scan_route(const VdaArgs& a) {
   const long long cta_comp = cta_scan * nc;
   const long long waves_scan = (cta_scan + slots - 1) / slots;
   const long long waves_comp = (cta_comp + slots - 1) / slots;
-  const long long cost_chunk = waves_comp * 2LL * (a.C - 1) + waves_scan * nc;
+  const long long cost_chunk = waves_comp * (2LL * a.C - 1) + waves_scan * nc;
   const long long cost_direct = waves_scan * (long long)a.T;
   return cost_direct <= cost_chunk;
 }
@@ -589,7 +650,7 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     kern<<<dim3(D / 32, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.alpha, a.FS, a.GS, B, H, T, a.C,
-                                                  a.init_scale);
+                                                  a.init_scale, a.frozen);
     return cudaGetLastError();
   }
   {
@@ -597,7 +658,8 @@ static cudaError_t launch_vda_states_t(const VdaArgs& a, cudaStream_t st) {
     auto kern = vda_chunk_compose_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3((D / 32) * nc, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.CM, a.CR, B, H, T, a.C);
+    kern<<<dim3((D / 32) * nc, H, 2 * B), 256, sm, st>>>(a.Mf, a.Rf, a.alpha, a.CM, a.CR, B, H,
+                                                         T, a.C, a.frozen);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {

@@ -3,10 +3,12 @@
 // "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
 // Generation": per frame, the statistics A_t = beta K_t^T K_t and
 // W_t = beta K_t^T V_t (Video Delta Attention, frame statistics), then the
-// inverse of (I + A_t) in key-channel space and the transition / injection
-// terms M_t = (I + A_t)^-1 Diag(alpha_t), R_t = (I + A_t)^-1 W_t
-// (implementation section, "Small-matrix inverse": Gauss-Jordan elimination
-// held in registers, FP32).
+// inverse X_t = (I + A_t)^-1 in key-channel space (implementation section,
+// "Small-matrix inverse": Gauss-Jordan elimination held in registers, FP32).
+// The frame update is S_t = X_t (Diag(alpha_t) S_{t-1} + W_t); this kernel
+// writes X_t and W_t and leaves the product with X_t to the scan, which needs
+// one product per frame either way.  The text virtual frame writes its state
+// X_0 W_0.
 //
 // One CTA per (b, h, frame); frame 0 is the text virtual frame.
 //   warp 0      TMA producer: 64-token tiles of K and V (bf16, 5-D maps
@@ -17,11 +19,11 @@
 //   all warps   epilogue: D -> shared memory (I + beta A, beta W), then the
 //               in-place Gauss-Jordan inversion of I + beta A with each thread
 //               holding a (d/16) x (d/16) block in registers (one barrier per
-//               pivot), then R = X W and M = X Diag(alpha) on CUDA cores (FP32).
+//               pivot); X and beta W out (text frame: X beta W on CUDA cores).
 // For d = 64 the MMA computes [K|V]^T [K|V] (M = N = 128) and keeps the first
-// 64 rows.  Anchor frames write M = Diag(alpha), R = 0 and exit.
-// Frozen-state rule (comparison mode): X = I - beta A without the inversion,
-// M = X Diag(alpha) and R = beta W.
+// 64 rows.  Anchor frames write X = I, W = 0 and exit.
+// Frozen-state rule (comparison mode): X = I - beta A without the inversion
+// and W = beta W; its update is S_t = X_t Diag(alpha_t) S_{t-1} + W_t.
 // Per-token write gates: warps 2-7 turn every landed bf16 tile into an exact
 // fp16 copy (the A operand, in place) and into beta_i-scaled fp16 hi and lo
 // parts (two B operands: beta*x = hi + lo to ~22 bits); two MMA chains
@@ -66,12 +68,11 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   float* Mo = Mout + (bh * (T + 1) + f) * mat;
   float* Ro = Rout + (bh * (T + 1) + f) * mat;
   const int t = f - 1;
-  const float* al = (alpha != nullptr && f >= 1) ? alpha + (bh * T + t) * D : nullptr;
 
-  if (f >= 1 && (t == 0 || t == T - 1)) {  // anchor: decay only, no write
+  if (f >= 1 && (t == 0 || t == T - 1)) {  // anchor: no write (X = I, W = 0)
     for (int e = tid; e < D * D; e += blockDim.x) {
       const int i = e / D, j = e % D;
-      Mo[e] = (i == j) ? (al ? al[i] : 1.f) : 0.f;
+      Mo[e] = (i == j) ? 1.f : 0.f;
       Ro[e] = 0.f;
     }
     return;
@@ -308,21 +309,16 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
       buf ^= 1;
     }
   }
-  // ---- M = X Diag(alpha) (registers), X -> shared, R = X W ----
+  // ---- X (registers) -> Mout; video frames: beta W -> Rout; text frame:
+  // X -> shared, R = X beta W -> Rout (the text state) ----
 #pragma unroll
   for (int i = 0; i < BL; ++i) {
     float* dst = Mo + (size_t)(ty * BL + i) * D + tx * BL;
 #pragma unroll
-    for (int c = 0; c < BL; c += 4) {
-      float4 m4;
-      m4.x = a[i][c] * (al ? al[tx * BL + c] : 1.f);
-      m4.y = a[i][c + 1] * (al ? al[tx * BL + c + 1] : 1.f);
-      m4.z = a[i][c + 2] * (al ? al[tx * BL + c + 2] : 1.f);
-      m4.w = a[i][c + 3] * (al ? al[tx * BL + c + 3] : 1.f);
-      *reinterpret_cast<float4*>(dst + c) = m4;
-    }
+    for (int c = 0; c < BL; c += 4)
+      *reinterpret_cast<float4*>(dst + c) = make_float4(a[i][c], a[i][c + 1], a[i][c + 2], a[i][c + 3]);
   }
-  if (frozen) {  // R = beta W (uniform over the CTA)
+  if (frozen || f >= 1) {  // R = beta W (uniform over the CTA)
 #pragma unroll
     for (int i = 0; i < BL; ++i) {
       float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
