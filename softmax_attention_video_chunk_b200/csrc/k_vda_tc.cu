@@ -16,10 +16,11 @@
 //   warp 1      MMA issuer: [K | V]^T-shaped products on tcgen05, both
 //               operands MN-major straight from the TMA tiles:
 //               D[128 x 2d] += K_t^T [K_t | V_t]  (FP32 in TMEM);
-//   all warps   epilogue: D -> shared memory (I + beta A, beta W), then the
-//               in-place Gauss-Jordan inversion of I + beta A with each thread
-//               holding a (d/16) x (d/16) block in registers (one barrier per
-//               pivot); X and beta W out (text frame: X beta W on CUDA cores).
+//   all warps   epilogue: D -> I + beta A in shared memory and beta W straight
+//               to Rout, then the in-place Gauss-Jordan inversion of I + beta A
+//               with each thread holding a (d/16) x (d/16) block in registers
+//               (one barrier per pivot); X out (text frame: X beta W on CUDA
+//               cores, W read back from Rout).
 // For d = 64 the MMA computes [K|V]^T [K|V] (M = N = 128) and keeps the first
 // 64 rows.  Anchor frames write X = I, W = 0 and exit.
 // Frozen-state rule (comparison mode): X = I - beta A without the inversion
@@ -39,7 +40,7 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* b
                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box);
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
 vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v,
                     const __grid_constant__ CUtensorMap map_tk,
@@ -58,7 +59,6 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   const int SSTR = beta_tok ? 3 * STB : STB;  // stage stride
   constexpr int NN = 2 * D;               // MMA N (columns of D)
   constexpr int SD = D + 1;               // padded row stride of I + beta A, then X
-  constexpr int SDW = D + 4;              // row stride of beta W (float4-aligned rows)
   constexpr int BL = D / 16;              // register block edge per thread
 
   const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -88,14 +88,14 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  // phase 1: TMA ring; phase 2 (after the MMAs): the two FP32 matrices
-  uint8_t* stages = smem;
-  float* Ash = (float*)smem;           // [D][SD]  I + beta A, then X
-  float* Wsh = Ash + D * SD;           // [D][SDW] beta W
-  constexpr int MATB = (D * SD + D * SDW) * 4;
-  constexpr int RING = 6 * STB;  // the larger of 3 x STB and 2 x 3 x STB
-  constexpr int BIG = (RING > MATB) ? RING : MATB;
-  uint64_t* full = (uint64_t*)(smem + ((BIG + 1023) & ~1023));
+  // the first 1 KB: barriers; then phase 1: the TMA ring (3 x STB, or
+  // 2 x 3 x STB with per-token gates); phase 2 (after the MMAs): I + beta A,
+  // inverted in place.  beta W goes from TMEM straight to Rout.  With per-frame
+  // gates this is under 100 KB, so two CTAs share an SM and one's inversion
+  // overlaps the other's loads and MMAs.
+  uint64_t* full = (uint64_t*)smem;
+  uint8_t* stages = smem + 1024;
+  float* Ash = (float*)stages;         // [D][SD]  I + beta A, then X
   uint64_t* empty = full + 3;
   uint64_t* conv_full = empty + 3;   // per-token gates: operands prepared
   uint64_t* acc_full = conv_full + 3;
@@ -223,7 +223,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
   // ---- epilogue: D -> shared (all warps) ----
   bool have = true;
   if (nst > 0) have = ptx::wait_bounded(acc_full, 0, abort_flag, status, kDevTimeout);
-  __syncthreads();  // every MMA done reading the stages: reuse them for Ash / Wsh
+  __syncthreads();  // every MMA done reading the stages: reuse them for Ash
   ptx::tc_fence_after();
   {
     const int q = warp & 3, part = warp >> 2;  // part 0: A columns, 1: W columns
@@ -247,14 +247,19 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
         for (int e = 0; e < 32; ++e) r[e] = 0u;
       }
       if (i < D) {
+        if (part == 0) {  // I + beta A (VDA), or I - beta A (frozen-state rule)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int j = 32 * c + e;
-          const float x = bt * __uint_as_float(r[e]);
-          if (part == 0)  // I + beta A (VDA), or I - beta A (frozen-state rule)
+          for (int e = 0; e < 32; ++e) {
+            const int j = 32 * c + e;
+            const float x = bt * __uint_as_float(r[e]);
             Ash[i * SD + j] = (frozen ? -x : x) + (i == j ? 1.f : 0.f);
-          else
-            Wsh[i * SDW + j] = x;
+          }
+        } else {          // beta W: row i, columns 32 c .. 32 c + 31
+          float4* dst = reinterpret_cast<float4*>(Ro + (size_t)i * D + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(bt * __uint_as_float(r[4 * e]), bt * __uint_as_float(r[4 * e + 1]),
+                                 bt * __uint_as_float(r[4 * e + 2]), bt * __uint_as_float(r[4 * e + 3]));
         }
       }
     }
@@ -318,27 +323,18 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
     for (int c = 0; c < BL; c += 4)
       *reinterpret_cast<float4*>(dst + c) = make_float4(a[i][c], a[i][c + 1], a[i][c + 2], a[i][c + 3]);
   }
-  if (frozen || f >= 1) {  // R = beta W (uniform over the CTA)
-#pragma unroll
-    for (int i = 0; i < BL; ++i) {
-      float* dst = Ro + (size_t)(ty * BL + i) * D + tx * BL;
-      const float* src = Wsh + (ty * BL + i) * SDW + tx * BL;
-#pragma unroll
-      for (int c = 0; c < BL; c += 4)
-        *reinterpret_cast<float4*>(dst + c) = make_float4(src[c], src[c + 1], src[c + 2], src[c + 3]);
-    }
-    return;
-  }
+  if (frozen || f >= 1) return;  // Rout already holds beta W (uniform over the CTA)
   __syncthreads();
 #pragma unroll
   for (int i = 0; i < BL; ++i)
 #pragma unroll
     for (int c = 0; c < BL; ++c) Ash[(ty * BL + i) * SD + tx * BL + c] = a[i][c];
   __syncthreads();
-  // R = X W: thread (ty, tx) computes rows ty*BL .. +BL-1 and the column
-  // groups {4 tx .. 4 tx + 3} + 4 D/4 g for g < BL/4 (groups of four columns,
-  // D/4 apart), so that the sixteen threads of a row group read W as
-  // consecutive float4 (no shared-memory bank conflicts)
+  // Text frame: R = X (beta W), W read back from Rout (written by this CTA's
+  // epilogue before the inversion's barriers).  Thread (ty, tx) computes rows
+  // ty*BL .. +BL-1 and the column groups {4 tx .. 4 tx + 3} + 4 D/4 g for
+  // g < BL/4 (groups of four columns, D/4 apart), so that the sixteen threads
+  // of a row group read W as consecutive float4.
   constexpr int NGR = BL / 4;
   float acc[BL][BL];
 #pragma unroll
@@ -352,7 +348,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
     for (int i = 0; i < BL; ++i) xv[i] = Ash[(ty * BL + i) * SD + l];
 #pragma unroll
     for (int g = 0; g < NGR; ++g) {
-      const float4 w4 = *reinterpret_cast<const float4*>(Wsh + l * SDW + g * (D / NGR) + tx * 4);
+      const float4 w4 = *reinterpret_cast<const float4*>(Ro + (size_t)l * D + g * (D / NGR) + tx * 4);
       wv[4 * g] = w4.x;
       wv[4 * g + 1] = w4.y;
       wv[4 * g + 2] = w4.z;
@@ -363,6 +359,7 @@ vda_frame_tc_kernel(const __grid_constant__ CUtensorMap map_k,
 #pragma unroll
       for (int c = 0; c < BL; ++c) acc[i][c] = fmaf(xv[i], wv[c], acc[i][c]);
   }
+  __syncthreads();  // every thread has read W before R overwrites it
 #pragma unroll
   for (int i = 0; i < BL; ++i) {
     float* dst = Ro + (size_t)(ty * BL + i) * D + tx * 4;
@@ -397,10 +394,10 @@ static cudaError_t launch_frame_tc_t(const VdaArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   constexpr int SD = D + 1;
-  const size_t stage_bytes = 6 * (size_t)(D / 32) * 64 * 128;
-  const size_t mat_bytes = 2 * (size_t)D * SD * 4;
-  const size_t big = ((stage_bytes > mat_bytes ? stage_bytes : mat_bytes) + 1023) & ~(size_t)1023;
-  const size_t sm = 1024 + big + 128;
+  // alignment slack + barriers (1 KB) + the larger of the TMA ring and I + beta A
+  const size_t stage_bytes = (a.beta_tok ? 6 : 3) * (size_t)(D / 32) * 64 * 128;
+  const size_t mat_bytes = (size_t)D * SD * 4;
+  const size_t sm = 1024 + 1024 + (stage_bytes > mat_bytes ? stage_bytes : mat_bytes);
   auto kern = vda_frame_tc_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
