@@ -479,16 +479,29 @@ vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf
       for (int r = 0; r < RT; ++r)
 #pragma unroll
         for (int m = 0; m < 4; ++m) acc[r][m] = 0.f;
+      // X_t is symmetric (the inverse of the symmetric I + beta A_t; the
+      // frozen rule's I - beta A_t is symmetric too), so X_t[i][l] is read as
+      // X_t[l][i]: this thread's RT rows at column l are RT consecutive floats
+      // of row l, one vector load instead of RT scalar ones
 #pragma unroll 4
       for (int l = 0; l < D; ++l) {
         const float4 sv = *reinterpret_cast<const float4*>(Ss + l * 32 + tx * 4);
+        float xa[RT];
+        if constexpr (RT == 4) {
+          const float4 x4 = *reinterpret_cast<const float4*>(Ms + l * SD + ty * RT);
+          xa[0] = x4.x; xa[1] = x4.y; xa[2] = x4.z; xa[3] = x4.w;
+        } else if constexpr (RT == 2) {
+          const float2 x2 = *reinterpret_cast<const float2*>(Ms + l * SD + ty * RT);
+          xa[0] = x2.x; xa[1] = x2.y;
+        } else {
+          xa[0] = Ms[l * SD + ty];
+        }
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-          const float a = Ms[(ty * RT + r) * SD + l];
-          acc[r][0] = fmaf(a, sv.x, acc[r][0]);
-          acc[r][1] = fmaf(a, sv.y, acc[r][1]);
-          acc[r][2] = fmaf(a, sv.z, acc[r][2]);
-          acc[r][3] = fmaf(a, sv.w, acc[r][3]);
+          acc[r][0] = fmaf(xa[r], sv.x, acc[r][0]);
+          acc[r][1] = fmaf(xa[r], sv.y, acc[r][1]);
+          acc[r][2] = fmaf(xa[r], sv.z, acc[r][2]);
+          acc[r][3] = fmaf(xa[r], sv.w, acc[r][3]);
         }
       }
       if (frozen) {
