@@ -151,7 +151,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 2;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* p_half = drain + 1;  // first 64 keys of P_j stored
+  uint32_t* tmem_slot = (uint32_t*)(p_half + 2);
   int* abort_flag = (int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -191,6 +192,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     for (int j = 0; j < 2; ++j) {
       ptx::mbar_init(s_full + j, 1);
       ptx::mbar_init(p_full + j, 128);
+      ptx::mbar_init(p_half + j, 128);
       ptx::mbar_init(o_done + j, 1);
     }
     ptx::mbar_init(drain, 1);
@@ -266,15 +268,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         }
         ptx::mma_commit(s_full + j);
       };
-      auto issue_PV = [&](int j, int st, bool first) {
+      // O_j += P_j V over key slices kk0 .. kk1-1 (16 keys each); the first
+      // half runs as soon as the softmax warps have stored P's first 64 keys
+      auto issue_PV = [&](int j, int st, bool first, int kk0, int kk1) {
         const uint32_t d = tmem + 256 + j * D;
         const uint32_t pa = tmem + j * 128;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
+        for (int kk = kk0; kk < kk1; ++kk) {
           const uint64_t bd = ptx::sdesc_k_sw128(sVa + st * VT + (kk >> 2) * (D * 128) + (kk & 3) * 32);
           ptx::mma_ts(d, pa + kk * 8, bd, idO, (!first || kk > 0) ? 1u : 0u);
         }
+      };
+      auto issue_PV_tile = [&](int j, int st, bool first, uint32_t ph) -> bool {
+        if (!wait_bar(p_half + j, ph, ab)) return false;
+        ptx::tc_fence_after();
+        issue_PV(j, st, first, 0, kBK / 32);
+        if (!wait_bar(p_full + j, ph, ab)) return false;
+        ptx::tc_fence_after();
+        issue_PV(j, st, first, kBK / 32, kBK / 16);
         ptx::mma_commit(o_done + j);
+        return true;
       };
       bool ok = wait_bar(q_full, 0, ab) && wait_bar(k_full, 0, ab);
       if (ok) {
@@ -286,19 +299,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int st = i % NS, ph = (i / NS) & 1;
         const int st2 = (i + 1) % NS, ph2 = ((i + 1) / NS) & 1;
         if (!(ok = wait_bar(v_full + st, ph, ab))) break;
-        if (!(ok = wait_bar(p_full + 0, i & 1, ab))) break;
-        ptx::tc_fence_after();
-        issue_PV(0, st, i == 0);
+        if (!(ok = issue_PV_tile(0, st, i == 0, i & 1))) break;
         if (i + 1 < n_kv) {
           if (!(ok = wait_bar(k_full + st2, ph2, ab))) break;
           ptx::tc_fence_after();
           issue_S(0, st2);
         }
-        if (has1) {
-          if (!(ok = wait_bar(p_full + 1, i & 1, ab))) break;
-          ptx::tc_fence_after();
-          issue_PV(1, st, i == 0);
-        }
+        if (has1 && !(ok = issue_PV_tile(1, st, i == 0, i & 1))) break;
         ptx::mma_commit(kv_empty + st);
         if (has1 && i + 1 < n_kv) issue_S(1, st2);
       }
@@ -392,6 +399,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             uint32_t (&rb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
             ptx::tmem_ld32(tS + 64 * half, ra);
             ptx::tmem_ld32(tS + 64 * half + 32, rb);
+            if (half == 1) {  // P's first 64 keys are stored: PV may start on them
+              ptx::tmem_wait_st();
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(p_half + j);
+            }
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -420,6 +432,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             uint32_t (&rb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
             ptx::tmem_ld32(tS + 64 * half, ra);
             ptx::tmem_ld32(tS + 64 * half + 32, rb);
+            if (half == 1) {  // P's first 64 keys are stored: PV may start on them
+              ptx::tmem_wait_st();
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(p_half + j);
+            }
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
