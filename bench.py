@@ -69,7 +69,7 @@ def work_model(cfg, out_bytes=4, text_keys=False):
 
 # DRAM bytes (read + write) of one attn_tc_kernel launch, from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum) of the 4-head copy of the
-# 768p workload: 1001.1 MB + 113.2 MB, scaled by the head count (the launch is
+# 768p workload: 987.6 MB + 113.5 MB, scaled by the head count (the launch is
 # one independent problem per head).  None for any other workload.
 ATTN_TRAFFIC_PER_HEAD = (987.616256e6 + 113.466368e6) / 4
 ATTN_TRAFFIC_SHAPES = {(75, 1536, 128)}
