@@ -10,11 +10,14 @@
 // that emits the transition and injection terms directly).
 //
 //   vda_frame_solve  : per frame, A_t = beta K^T K, W_t = beta K^T V, then
-//                      Gauss-Jordan on [I + A_t | Diag(alpha_t) | W_t] ->
-//                      M_t = (I + A_t)^-1 Diag(alpha_t), R_t = (I + A_t)^-1 W_t.
-//                      Frame index 0 is the text "virtual frame" (R_0 = S_text);
-//                      anchor frames emit M = Diag(alpha), R = 0 (excluded from
-//                      both scans, decay kept).
+//                      Gauss-Jordan on [I + A_t | I] -> X_t = (I + A_t)^-1;
+//                      writes X_t and W_t (the affine map of frame t is
+//                      S -> X_t (Diag(alpha_t) S + W_t)).  Frame index 0 is the
+//                      text "virtual frame" (it writes S_text = X_0 W_0); anchor
+//                      frames emit X = I, W = 0 (excluded from both scans, decay
+//                      kept).
+//   vda_frame_scan   : for short clips, the scan over frames directly, keeping
+//                      only the chunk-boundary states.
 //   vda_chunk_compose: per chunk and direction, the product of its frames'
 //                      affine maps in scan order.
 //   vda_chunk_scan   : per (b, h, direction, 32-column slice of S), the
@@ -422,7 +425,7 @@ vda_frame_scan_kernel(const float* __restrict__ Mf, const float* __restrict__ Rf
       OUT[(bh * (nc + 1) + k0) * mat + i * D + cb + j] = Ss[q];
     }
   }
-  // M_t of the next frame is loaded into registers (D*D/4/256 float4 per
+  // X_t of the next frame is loaded into registers (D*D/4/256 float4 per
   // thread, all in flight at once) while the current frame's product runs
   constexpr int NV = D * D / 4 / 256;
   float4 mv[NV];
