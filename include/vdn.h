@@ -191,7 +191,8 @@ VDN_API vdn_status vdn_hybrid_attn_fwd(const vdn_params *p, const void *q, const
  * frames) or 3 (frame statistics + solve, chunk composition, chunk scan): the
  * library picks the route from the shape and the device's SM count unless
  * VDN_FLAG_SCAN_FRAMES / VDN_FLAG_SCAN_CHUNKS forces it.  Then, on the
- * tensor-core path: V^T conversion, Softmax, readout, W^T conversion and the
+ * tensor-core path: V^T conversion (a second one for the text values when
+ * VDN_FLAG_TEXT_SOFTMAX adds text keys), Softmax, readout, W^T conversion and the
  * GEMM (with VDN_FLAG_PROJ_MXFP8: the quantisation of W^T and the block-
  * scaled GEMM, x arriving quantised from the epilogues); on the CUDA-core
  * path: Softmax, readout, RMS factors, projection.

@@ -715,8 +715,9 @@ vdn_status vdn_forward_launches(const vdn_params* p, int* launches) {
   va.B = p->B; va.H = p->H; va.T = p->T; va.D = p->d_k; va.C = p->chunk;
   va.scan_mode = (p->flags & VDN_FLAG_SCAN_FRAMES) ? 1 : ((p->flags & VDN_FLAG_SCAN_CHUNKS) ? 2 : 0);
   int n = vda_frame_scan_route(va) ? 2 : 3;
-  if (use_tc(*p))
-    n += 4 + ((p->flags & VDN_FLAG_PROJ_MXFP8) ? 2 : 1);
+  if (use_tc(*p))  // V^T conversion (text V^T too when text keys join), Softmax, readout, W^T, GEMM
+    n += 4 + ((p->flags & VDN_FLAG_PROJ_MXFP8) ? 2 : 1) +
+         (((p->flags & VDN_FLAG_TEXT_SOFTMAX) && p->n_text > 0) ? 1 : 0);
   else
     n += 4;
   *launches = n;

@@ -322,6 +322,9 @@ def test_mxfp8_projection_needs_the_tensor_core_path():
     ((1, 2, 15, 16, 64, 8), "bf16", 0, 8),
     # one chunk: the frame scan (2 products) beats composition (8 + 1)
     ((1, 2, 2, 16, 64, 8), "bf16", 0, 7),
+    # text keys in the Softmax: the text values get their own V^T conversion
+    ((1, 24, 75, 1536, 128, 512), "bf16", vdn.FLAG_TEXT_SOFTMAX, 8),
+    ((1, 24, 75, 1536, 128, 0), "bf16", vdn.FLAG_TEXT_SOFTMAX, 7),
     # CUDA-core path: states (2 or 3), Softmax, readout, RMS factors, projection
     ((1, 24, 75, 1536, 128, 512), "f32", 0, 6),
     ((1, 2, 15, 16, 64, 8), "bf16", vdn.FLAG_SIMT, 7),

@@ -36,6 +36,7 @@ CASES = [
     ("frames", dict(T=20, N=64, H=2, d=128, n_text=16), vdn.FLAG_SCAN_FRAMES),
     ("chunks", dict(T=20, N=64, H=2, d=128, n_text=16), vdn.FLAG_SCAN_CHUNKS),
     ("mxfp8", dict(T=12, N=64, H=2, d=64, n_text=16), vdn.FLAG_PROJ_MXFP8),
+    ("text_softmax", dict(T=12, N=64, H=2, d=64, n_text=16), vdn.FLAG_TEXT_SOFTMAX),
     ("simt", dict(T=12, N=64, H=2, d=64, n_text=16), vdn.FLAG_SIMT),
 ]
 
