@@ -39,19 +39,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Non-blocking test of a phase (never suspends the thread): several of these
-// can be in flight at once, unlike a chain of blocking waits.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -174,49 +161,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       VDN_TM_IREGS32(r)
       : "memory");
 }
-// Same as tmem_ld32 / tmem_st32 on 32 consecutive elements arr[off .. off+31]
-// of a register array (compile-time indices keep the array in registers).
-#define VDN_R32(a, o)                                                                          \
-  a[o + 0], a[o + 1], a[o + 2], a[o + 3], a[o + 4], a[o + 5], a[o + 6], a[o + 7], a[o + 8],    \
-      a[o + 9], a[o + 10], a[o + 11], a[o + 12], a[o + 13], a[o + 14], a[o + 15], a[o + 16],   \
-      a[o + 17], a[o + 18], a[o + 19], a[o + 20], a[o + 21], a[o + 22], a[o + 23], a[o + 24],  \
-      a[o + 25], a[o + 26], a[o + 27], a[o + 28], a[o + 29], a[o + 30], a[o + 31]
-__device__ __forceinline__ void tmem_ld32_r(
-    uint32_t taddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t& r4,
-    uint32_t& r5, uint32_t& r6, uint32_t& r7, uint32_t& r8, uint32_t& r9, uint32_t& r10,
-    uint32_t& r11, uint32_t& r12, uint32_t& r13, uint32_t& r14, uint32_t& r15, uint32_t& r16,
-    uint32_t& r17, uint32_t& r18, uint32_t& r19, uint32_t& r20, uint32_t& r21, uint32_t& r22,
-    uint32_t& r23, uint32_t& r24, uint32_t& r25, uint32_t& r26, uint32_t& r27, uint32_t& r28,
-    uint32_t& r29, uint32_t& r30, uint32_t& r31) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3), "=r"(r4), "=r"(r5), "=r"(r6), "=r"(r7),
-        "=r"(r8), "=r"(r9), "=r"(r10), "=r"(r11), "=r"(r12), "=r"(r13), "=r"(r14), "=r"(r15),
-        "=r"(r16), "=r"(r17), "=r"(r18), "=r"(r19), "=r"(r20), "=r"(r21), "=r"(r22),
-        "=r"(r23), "=r"(r24), "=r"(r25), "=r"(r26), "=r"(r27), "=r"(r28), "=r"(r29),
-        "=r"(r30), "=r"(r31)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32_r(
-    uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3, uint32_t r4, uint32_t r5,
-    uint32_t r6, uint32_t r7, uint32_t r8, uint32_t r9, uint32_t r10, uint32_t r11, uint32_t r12,
-    uint32_t r13, uint32_t r14, uint32_t r15, uint32_t r16, uint32_t r17, uint32_t r18,
-    uint32_t r19, uint32_t r20, uint32_t r21, uint32_t r22, uint32_t r23, uint32_t r24,
-    uint32_t r25, uint32_t r26, uint32_t r27, uint32_t r28, uint32_t r29, uint32_t r30,
-    uint32_t r31) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7), "r"(r8), "r"(r9),
-      "r"(r10), "r"(r11), "r"(r12), "r"(r13), "r"(r14), "r"(r15), "r"(r16), "r"(r17), "r"(r18),
-      "r"(r19), "r"(r20), "r"(r21), "r"(r22), "r"(r23), "r"(r24), "r"(r25), "r"(r26), "r"(r27),
-      "r"(r28), "r"(r29), "r"(r30), "r"(r31)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -297,41 +241,6 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;             // 128-byte swizzle
   return d;
-}
-
-// The same descriptor split into its two 32-bit words: the low word holds the
-// start address (>> 4) and the leading byte offset, the high word the stride
-// byte offset, version and swizzle mode, which are the same for every K-major
-// 128-byte-swizzled operand.  Moving the start address by `off` bytes (a
-// multiple of 16 inside shared memory) adds off >> 4 to the low word, so an
-// MMA issue loop can step through K with one 32-bit add per operand.
-__device__ __forceinline__ uint32_t sdesc_k_sw128_lo(uint32_t saddr) {
-  return ((saddr & 0x3FFFFu) >> 4) | (1u << 16);
-}
-constexpr uint32_t kSdescKSw128Hi = (1024u >> 4) | (1u << 14) | (2u << 29);
-
-// D[tmem] (+)= A[smem] * B[smem]^T from the low descriptor words.
-__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "mov.b64 da, {%1, %5};\n\t"
-      "mov.b64 db, {%2, %5};\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescKSw128Hi)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]^T from the low descriptor word of B.
-__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "mov.b64 db, {%2, %5};\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSdescKSw128Hi)
-      : "memory");
 }
 
 // Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle: rows of
