@@ -22,9 +22,9 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _cfg():
+def _cfg(H=4):
     from synth import CONFIGS
-    return CONFIGS["tiny_f32"].replace(H=4)
+    return CONFIGS["tiny_f32"].replace(H=H)
 
 
 def _oracle_operand(cfg):
@@ -63,7 +63,7 @@ def _oracle_fwd(cfg):
     return fwd
 
 
-def _rank(rank, world, port, out, alpha):
+def _rank(rank, world, port, out, alpha, gates="const", H=4):
     import datetime
 
     import torch.distributed as dist
@@ -75,8 +75,8 @@ def _rank(rank, world, port, out, alpha):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=120))
     try:
-        cfg = _cfg()
-        inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None)
+        cfg = _cfg(H)
+        inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None, gates=gates)
         Ls = cfg.L // world
         tok = slice(rank * Ls, (rank + 1) * Ls)
         y = ulysses.ulysses_forward(
@@ -91,15 +91,17 @@ def _rank(rank, world, port, out, alpha):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,alpha", [(2, False), (4, True)])
-def test_head_sharded_forward_equals_unsharded(world, alpha):
+@pytest.mark.parametrize("world,alpha,gates,H", [(2, False, "const", 4), (4, True, "random", 4),
+                                                 (3, True, "random", 6)])
+def test_head_sharded_forward_equals_unsharded(world, alpha, gates, H):
     from synth import make_inputs
-    cfg = _cfg()
+    cfg = _cfg(H)
     with mp.Manager() as m:
         out = m.dict()
-        mp.spawn(_rank, args=(world, _free_port(), out, alpha), nprocs=world, join=True)
+        mp.spawn(_rank, args=(world, _free_port(), out, alpha, gates, H), nprocs=world,
+                 join=True)
         got = out["y"]
-    inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None)
+    inp = make_inputs(cfg, alpha_range=(0.8, 1.0) if alpha else None, gates=gates)
     want = _oracle_fwd(cfg)(inp["q"], inp["k"], inp["v"], inp["beta"], inp["text_k"],
                             inp["text_v"], inp["W_soft"], inp["W_lin"], inp["gates"], cfg.T,
                             alpha=inp["alpha"]).numpy()
