@@ -459,13 +459,18 @@ def run_ours(args, cfg):
 
 
 def main():
+    from synth import CONFIGS
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="768p_bf16")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of the job (one replica per rank under torchrun)")
+    ap.add_argument("--steps", type=int, default=10, help="timed forwards")
+    ap.add_argument("--warmup", type=int, default=3, help="untimed forwards before them")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="ours: the library; reference: the float64 oracle on a sample")
+    ap.add_argument("--config", default="768p_bf16",
+                    help="workload: " + ", ".join(sorted(CONFIGS)))
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the timed oracle sample on the host cores")
     ap.add_argument("--text-softmax", action="store_true",
                     help="video queries also attend all text tokens in the Softmax branch")
     ap.add_argument("--beta-per-token", action="store_true",
@@ -479,7 +484,6 @@ def main():
     ap.add_argument("--alpha", action="store_true",
                     help="channel-wise decay gate alpha ~ U[0.9, 1] instead of none")
     args = ap.parse_args()
-    from synth import CONFIGS
     cfg = CONFIGS[args.config]
     if args.impl == "reference":
         return run_reference(args, cfg)
